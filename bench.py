@@ -1,0 +1,413 @@
+"""Benchmark of the KATA chunked-state causal forward (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one kata_fwd_chunked call over one batch of the long-context
+workload (B=1, H=16, T=131072, d_k=32, d_v=64, C=128, bf16 inputs, fp32
+accumulation; PSD feature), inputs resident in HBM. With N > 1 (launched by
+torch.distributed.run) every rank runs its own batch (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+
+The per-step input (805 MB) is larger than the 126 MB L2, so no L2 flush is
+needed between steps.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KATA causal fwd tokens/sec at T=131072 (chunked) and % of tensor/HBM roofline"
+UNIT = "tokens/s"
+NOMINAL_FP32_TFLOPS_PER_SM_GHZ = 128 * 2 / 1000.0   # 128 FP32 lanes x FMA, per GHz, in TFLOP/s
+
+# Which roofline each of the library's kernels is held to.
+#   tensor: bf16 tensor-core contraction;  alu: fp32 FFMA on the CUDA cores;
+#   hbm: streaming kernel.
+KERNEL_BOUND = {
+    "simt_segment_pass": "alu",
+    "simt_segment_increment": "alu",
+    "simt_quadratic": "alu",
+    "simt_decode": "hbm",
+}
+
+
+def algorithmic_per_token_head(d_k, d_v, C, feature="psd"):
+    """(flops, bytes) the chunked forward must do per token-head: the causal
+    half of the intra-chunk block, the state update and the readout; bf16
+    q, k, v read once and o written once."""
+    D = d_k * (d_k + 1) // 2 if feature == "psd" else d_k + 1
+    intra = (C + 1) / 2 * (2 * d_k + 2 * d_v + 2)
+    update = 2 * D * d_v + D
+    readout = 2 * D * d_v + 2 * D
+    return intra + update + readout, (2 * d_k + d_v) * 2 + d_v * 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "sm_max_mhz": p.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kernelized_linear_attention_kata_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("source_sha") != source_hash():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        rows = []
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7],
+                             "sw_power": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        loaded = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and --impl reference arm)
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_sample(w, budget_s):
+    """Time the oracle's chunked form, as it stands, on whole heads of the
+    workload (full length T), head after head until `budget_s` seconds of CPU
+    work have been spent. Returns (tokens/s, description of the sample)."""
+    import oracle as O
+    from kernelized_linear_attention_kata_b200 import workloads as W
+
+    if w.name not in _ORACLE_INPUTS:
+        q, k, v = W.make_inputs(w)
+        _ORACLE_INPUTS[w.name] = (W.to_f64_numpy(q), W.to_f64_numpy(k), W.to_f64_numpy(v))
+    qn, kn, vn = _ORACLE_INPUTS[w.name]
+    token_heads = 0
+    heads = 0
+    t0 = time.perf_counter()
+    for bh in range(w.B * w.H):
+        b, h = divmod(bh, w.H)
+        O.forward_chunked(qn[b, h], kn[b, h], vn[b, h], w.C, w.feature)
+        token_heads += w.T
+        heads += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return token_heads / w.H / dt, (
+        f"oracle forward_chunked (fp64 numpy) on {heads} of {w.B * w.H} heads x {w.T} tokens of "
+        f"{w.name} in {dt:.1f} s; tokens/s = token-heads processed / H / s")
+
+
+def run_reference(args, rank, world):
+    from kernelized_linear_attention_kata_b200 import workloads as W
+    if rank != 0:
+        return 0
+    w = W.WORKLOADS[args.workload]
+    budget = args.ref_step_budget or max(0.5, 150.0 / (args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, budget_s=budget)
+    vals = []
+    sample = ""
+    for _ in range(args.steps):
+        v, sample = oracle_sample(w, budget_s=budget)
+        vals.append(v)
+    value = statistics.mean(vals)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_k": w.d_k, "d_v": w.d_v,
+            "C": w.C, "feature": w.feature, "form": "chunked (segmented scan carry)",
+            "l2": "inputs larger than L2 (no flush needed)", "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from kernelized_linear_attention_kata_b200 import api
+    from kernelized_linear_attention_kata_b200 import build as kbuild
+    from kernelized_linear_attention_kata_b200 import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    kbuild.build()
+    w = W.WORKLOADS[args.workload]
+    if args.T:
+        w = w.with_T(args.T)
+    dev = torch.device("cuda", local_rank)
+    # seeded synthetic inputs, generated on the device (one batch per rank)
+    from dataclasses import replace
+    w_rank = replace(w, seed=w.seed + 1000 * rank)
+    q, k, v = W.make_inputs(w_rank, device=dev)
+    o = torch.empty_like(v)
+    ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = api.kata_workspace_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        api.profile_enable(True)
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        prof = api.profile_read()
+        api.profile_enable(False)
+    ms = start.elapsed_time(end) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens_per_step = w.B * w.T
+    value = world * tokens_per_step / (ms / 1e3)
+
+    # roofline of the dominant kernel, timed live by the library's events
+    peaks = load_peaks()
+    dom = max(prof, key=lambda n: prof[n][1])
+    launches, dom_ms = prof[dom]
+    dom_avg_s = dom_ms / launches / 1e3
+    flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
+    token_heads = w.B * w.H * w.T
+    # achieved = the step's algorithmic work / one launch of the dominant kernel
+    per_launch_units = token_heads
+    bound = KERNEL_BOUND.get(dom, "tensor")
+    timed_s = ms * args.steps / 1e3
+    if bound == "hbm":
+        achieved = bytes_th * per_launch_units / dom_avg_s / 1e9
+        peak, unit, peak_kind = peaks["hbm_gbs"], "GB/s", peaks["source"]
+    elif bound == "alu":
+        achieved = flops_th * per_launch_units / dom_avg_s / 1e12
+        peak = 148 * NOMINAL_FP32_TFLOPS_PER_SM_GHZ * peaks["sm_max_mhz"] / 1000.0
+        unit, peak_kind = "TFLOP/s", "derived: 148 SMs x 128 FP32 FMA lanes x 2 x max SM clock"
+    else:
+        achieved = flops_th * per_launch_units / dom_avg_s / 1e12
+        sustained = timed_s > 1.0
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+        peak_kind = f"{peaks['source']} bf16 {'sustained' if sustained else 'burst'}"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": recorded_traffic(dom), "kernel": dom,
+                "kernel_ms": dom_ms / launches, "peak_kind": peak_kind,
+                "step_frac_of_tensor_or_hbm": None}
+    # whole-step fraction of the binding tensor/HBM roofline of the method
+    t_tensor = flops_th * token_heads / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = bytes_th * token_heads / (peaks["hbm_gbs"] * 1e9)
+    roofline["step_frac_of_tensor_or_hbm"] = max(t_tensor, t_hbm) / (ms / 1e3)
+    gpu_launches = sum(n for n, _ in prof.values())
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh = q.cpu().pin_memory()
+        kh = k.cpu().pin_memory()
+        vh = v.cpu().pin_memory()
+        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+
+        def e2e_step():
+            q.copy_(qh, non_blocking=True)
+            k.copy_(kh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws)
+            oh.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(2, min(args.steps, 10))
+        s2.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e2.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = s2.elapsed_time(e2) / n_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * tokens_per_step / (ms_e2e / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (q, k, v)),
+               "d2h_bytes_per_step": o.numel() * o.element_size(), "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, sample = oracle_sample(W.WORKLOADS[args.workload], budget_s=args.cpu_budget)
+        cpu = {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w) | {"parallelism": f"replicas x{world}"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+            "kernels": {n: {"launches": c, "avg_ms": t / c} for n, (c, t) in prof.items()},
+            "clocks": clocks.summary(), "token_heads_per_s": value * w.H,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long131k_bf16")
+    ap.add_argument("--T", type=int, default=0, help="override T (profiling a smaller case)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--ref-step-budget", type=float, default=0.0,
+                    help="seconds of oracle work per reference step (default: 150 s / (K + W))")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,201 @@
+/*
+ * kata.h -- C ABI of the KATA causal linear-attention library (CUDA, sm_100a).
+ *
+ * The method (Kernelized Linear Attention, "Kernelized Linear Attention:
+ * Breaking the Capacity Wall with Symmetric Cones", arXiv 2607.17419v1):
+ *
+ *   y_t = sum_{s<=t} w_ts v_s / sum_{s<=t} w_ts,
+ *   w_ts = <phi(q_t), phi(k_s)>.
+ *
+ * Normalised linear attention as an RNN with a fixed-size state ("線形注意"
+ * wiki page, definition); the rank-one PSD feature psi(u) = u u^T, whose
+ * weight is <q_t, k_s>^2 >= 0 (gist.science explainer, technical summary
+ * 2.2); the normaliser read as a convex output gate (same explainer, 2.1);
+ * the exact O(T) chunked-state form with an associative scan across chunks
+ * (same explainer, 2.3, and the arXiv abstract).
+ *
+ * Conventions common to every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    allocates no device memory; scratch is the caller's workspace.
+ *  - Layouts: q, k are [B, H, T, d_k]; v, o are [B, H, T, d_v]; row-major and
+ *    contiguous, element type `dtype` (o has the same type as q). States are
+ *    always fp32.
+ *  - Causal mask includes the diagonal (s <= t): y_1 = v_1.
+ *  - No temperature or 1/sqrt(d) scale is applied: pass q, k as they should
+ *    enter the inner product.
+ *  - Packed state layout, shape [B, H, D, d_v] for S and [B, H, D] for z:
+ *      PSD         : D = d_k (d_k + 1) / 2, row r <-> pair (i, j), i <= j,
+ *                    rows ordered row-major over i then j;
+ *                    S[r] = sum_s k_si k_sj v_s, z[r] = sum_s k_si k_sj
+ *                    (no factor 2: the readout applies the multiplicity 2
+ *                    of the off-diagonal pairs on the query side).
+ *      FIRST_ORDER : D = d_k + 1, row 0 is the constant feature 1, row 1 + i
+ *                    is k_i; weight 1 + <q_t, k_s>.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream). Argument errors are detected on the host and returned
+ *    before anything is launched. KATA_ERR_CUDA reports a launch error
+ *    (cudaGetLastError) and leaves outputs undefined.
+ *  - A row whose normaliser is not positive (for instance a query orthogonal
+ *    to every key it sees) yields a non-finite output. kata_fwd_chunked also
+ *    records this in its workspace; see kata_workspace_status.
+ *  - B, H or T equal to 0 is a valid empty problem: nothing is launched for
+ *    the outputs (S_out / z_out, when given, are zero-filled).
+ *
+ * Supported shapes (anything else returns KATA_ERR_UNSUPPORTED):
+ *    PSD          d_k in {16, 32}
+ *    FIRST_ORDER  d_k in {16, 32, 64}
+ *    d_v in {16, 32, 64};  C in {16, 32, 64, 128};  T >= 0;
+ *    T need not be a multiple of C (the last chunk is shorter).
+ */
+#ifndef KATA_H
+#define KATA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KATA_API __attribute__((visibility("default")))
+#else
+#define KATA_API
+#endif
+
+/* cudaStream_t without including the CUDA headers. */
+typedef struct CUstream_st *kata_stream_t;
+
+typedef enum {
+    KATA_OK = 0,
+    KATA_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, ...       */
+    KATA_ERR_UNSUPPORTED = 2,      /* shape / dtype / feature not built      */
+    KATA_ERR_WORKSPACE = 3,        /* workspace missing, too small, unaligned */
+    KATA_ERR_CUDA = 4,             /* a CUDA call or launch failed           */
+    KATA_ERR_NONPOSITIVE_NORMALISER = 5 /* device: some row had den <= 0     */
+} kata_status_t;
+
+typedef enum { KATA_DTYPE_F32 = 0, KATA_DTYPE_BF16 = 1 } kata_dtype_t;
+
+typedef enum { KATA_FEATURE_PSD = 0, KATA_FEATURE_FIRST_ORDER = 1 } kata_feature_t;
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+KATA_API int kata_version(void);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+KATA_API const char *kata_status_string(kata_status_t status);
+
+/* D, the number of state rows: d_k (d_k + 1) / 2 for PSD, d_k + 1 for
+ * FIRST_ORDER; 0 for an unknown feature or d_k <= 0. */
+KATA_API size_t kata_state_dim(int d_k, kata_feature_t feature);
+
+/*
+ * Workspace bytes kata_fwd_chunked needs for this problem on the CURRENT
+ * device (the segment split depends on its SM count). Returns 0 for a shape
+ * the library does not support. The workspace must be 256-byte aligned and
+ * must not be used by two calls that run concurrently.
+ */
+KATA_API size_t kata_fwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C,
+                                        kata_dtype_t dtype, kata_feature_t feature);
+
+/*
+ * Exact O(T) chunked-state causal forward (arXiv abstract: "exact O(T)
+ * chunked-state form"; explainer 2.3: chunk parallelism with an associative
+ * scan across chunks).
+ *
+ * For each chunk c of C tokens:
+ *   A     = (Q_c K_c^T)^2 masked to s <= t          (PSD; 1 + Q_c K_c^T for
+ *                                                   FIRST_ORDER)
+ *   Y_c   = (A V_c + phi_q(Q_c) S_c) / (A 1 + phi_q(Q_c) z_c)
+ *   S_c+1 = S_c + phi(K_c)^T V_c,  z_c+1 = z_c + phi(K_c)^T 1.
+ * The carry S_c is an exclusive scan of the per-chunk increments, computed
+ * per segment of chunks so the sequence is processed in parallel.
+ *
+ *   q, k, v, o         device, layouts above.
+ *   S_out, z_out       optional (may be NULL, independently): the final state
+ *                      after all T tokens, [B, H, D, d_v] and [B, H, D] fp32.
+ *   workspace          device, >= kata_fwd_chunked_workspace_bytes(...),
+ *                      256-byte aligned; contents on entry are ignored. On
+ *                      return (after the stream has run) it holds the device
+ *                      status word read by kata_workspace_status.
+ * Returns KATA_OK when the work was launched.
+ */
+KATA_API kata_status_t kata_fwd_chunked(const void *q, const void *k, const void *v, void *o,
+                               int B, int H, int T, int d_k, int d_v, int C,
+                               kata_dtype_t dtype, kata_feature_t feature,
+                               float *S_out, float *z_out,
+                               void *workspace, size_t workspace_bytes,
+                               kata_stream_t stream);
+
+/*
+ * The same forward with a SEQUENTIAL inter-chunk carry: one thread block per
+ * (b, h) walks its chunks in order (recurrence depth N_C = ceil(T/C)). This
+ * is the matched sequential linear-attention baseline that the arXiv
+ * abstract compares the associative scan against. Same arguments and
+ * results as kata_fwd_chunked; needs only the status header of the
+ * workspace (kata_fwd_chunked_workspace_bytes is always enough).
+ */
+KATA_API kata_status_t kata_fwd_chunked_sequential(const void *q, const void *k, const void *v, void *o,
+                                          int B, int H, int T, int d_k, int d_v, int C,
+                                          kata_dtype_t dtype, kata_feature_t feature,
+                                          float *S_out, float *z_out,
+                                          void *workspace, size_t workspace_bytes,
+                                          kata_stream_t stream);
+
+/*
+ * Flash-attention-style quadratic causal forward (explainer 2.3, operating
+ * point 1: O(T^2), no state is materialised). For each query block the key
+ * blocks up to the diagonal are visited; P = (Q K^T)^2 (or 1 + Q K^T) masked,
+ * O += P V, l += rowsum(P); finally O / l. No exponential and no running
+ * maximum are needed because the weights are polynomial and nonnegative.
+ * Same tensor layouts; no workspace.
+ */
+KATA_API kata_status_t kata_fwd_quadratic(const void *q, const void *k, const void *v, void *o,
+                                 int B, int H, int T, int d_k, int d_v,
+                                 kata_dtype_t dtype, kata_feature_t feature,
+                                 kata_stream_t stream);
+
+/*
+ * One-token recurrent decode step ("線形注意" definition: constant-time
+ * recurrent inference with a fixed-size state), batched over B x H heads:
+ *   S += phi(k) v^T,  z += phi(k),  y = phi_q(q)^T S / phi_q(q)^T z
+ * (update first, then read, so the current token is included exactly as in
+ * the forward).
+ *   q, k   device [B, H, d_k], dtype;  v, y device [B, H, d_v], dtype.
+ *   S, z   device fp32 [B, H, D, d_v] and [B, H, D], read and written in
+ *          place (packed layout above).
+ */
+KATA_API kata_status_t kata_decode_step(const void *q, const void *k, const void *v,
+                               float *S, float *z, void *y,
+                               int B, int H, int d_k, int d_v,
+                               kata_dtype_t dtype, kata_feature_t feature,
+                               kata_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the status word a kata_fwd_chunked(...)
+ * or kata_fwd_chunked_sequential(...) call left in `workspace`: KATA_OK, or
+ * KATA_ERR_NONPOSITIVE_NORMALISER if any row had a normaliser <= 0, or
+ * KATA_ERR_CUDA if the synchronisation or the copy failed.
+ */
+KATA_API kata_status_t kata_workspace_status(const void *workspace, kata_stream_t stream);
+
+/*
+ * Optional per-kernel device timing (CUDA events), for benchmarks. Not part
+ * of the method. kata_profile_enable(1) clears the counters and starts
+ * bracketing every kernel the library launches with two events recorded on
+ * the launch's stream; kata_profile_enable(0) stops. kata_profile_count and
+ * kata_profile_get synchronise on the recorded events, then report, per
+ * kernel name (static storage), the number of launches and their summed
+ * device time in milliseconds. Use from one host thread.
+ */
+KATA_API kata_status_t kata_profile_enable(int enable);
+KATA_API int kata_profile_count(void);
+KATA_API kata_status_t kata_profile_get(int index, const char **name, long long *launches,
+                                        double *total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KATA_H */

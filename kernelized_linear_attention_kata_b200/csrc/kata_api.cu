@@ -1,0 +1,243 @@
+// C ABI of the KATA library: argument validation, workspace layout and
+// kernel dispatch. Declarations and the full contract are in include/kata.h.
+#include "../../include/kata.h"
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+using namespace kata;
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;   // status word + padding
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool supported(int d_k, int d_v, int C, kata_dtype_t dtype, kata_feature_t feature) {
+  if (dtype != KATA_DTYPE_F32 && dtype != KATA_DTYPE_BF16) return false;
+  if (feature == KATA_FEATURE_PSD) {
+    if (d_k != 16 && d_k != 32) return false;
+  } else if (feature == KATA_FEATURE_FIRST_ORDER) {
+    if (d_k != 16 && d_k != 32 && d_k != 64) return false;
+  } else {
+    return false;
+  }
+  if (d_v != 16 && d_v != 32 && d_v != 64) return false;
+  if (C != 0 && C != 16 && C != 32 && C != 64 && C != 128) return false;
+  return true;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// Segment split of the chunked forward: G segments of `chunks_per_seg`
+// chunks per (b, h), sized so that B*H*G blocks fill the SMs once.
+struct Split {
+  int G;
+  int seg_len;   // tokens per segment (a multiple of C)
+};
+
+Split segment_split(long long BH, int T, int C, int sms, bool sequential) {
+  const int n_chunks = T <= 0 ? 0 : (T + C - 1) / C;
+  if (sequential || n_chunks <= 1 || BH >= sms) return {1, n_chunks * C};
+  long long G = sms / BH;
+  if (G < 1) G = 1;
+  if (G > n_chunks) G = n_chunks;
+  const int per = (int)((n_chunks + G - 1) / G);
+  const int Gr = (n_chunks + per - 1) / per;
+  return {Gr, per * C};
+}
+
+size_t workspace_bytes_for(long long BH, int D, int d_v, const Split &sp) {
+  const size_t agg = (size_t)BH * (size_t)sp.G * (size_t)D * (size_t)(d_v + 1) * sizeof(float);
+  return kHeaderBytes + align_up(agg, kAlign);
+}
+
+// Calls F::template run<DK, DV, FEAT>() for the runtime (d_k, d_v, feature).
+template <typename F>
+kata_status_t dispatch_shape(int d_k, int d_v, kata_feature_t feature, F &&f) {
+#define KATA_DV_CASES(DK, FEAT)                                         \
+  switch (d_v) {                                                        \
+    case 16: return f.template operator()<DK, 16, FEAT>();              \
+    case 32: return f.template operator()<DK, 32, FEAT>();              \
+    case 64: return f.template operator()<DK, 64, FEAT>();              \
+    default: return KATA_ERR_UNSUPPORTED;                               \
+  }
+  if (feature == KATA_FEATURE_PSD) {
+    if (d_k == 16) { KATA_DV_CASES(16, kPSD) }
+    if (d_k == 32) { KATA_DV_CASES(32, kPSD) }
+  } else {
+    if (d_k == 16) { KATA_DV_CASES(16, kFirstOrder) }
+    if (d_k == 32) { KATA_DV_CASES(32, kFirstOrder) }
+    if (d_k == 64) { KATA_DV_CASES(64, kFirstOrder) }
+  }
+#undef KATA_DV_CASES
+  return KATA_ERR_UNSUPPORTED;
+}
+
+struct ChunkedRun {
+  kata_dtype_t dtype;
+  ChunkedLaunch a;
+  template <int DK, int DV, int FEAT> kata_status_t operator()() {
+    cudaError_t e = dtype == KATA_DTYPE_F32 ? simt_chunked<DK, DV, FEAT, float>(a)
+                                            : simt_chunked<DK, DV, FEAT, __nv_bfloat16>(a);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+  }
+};
+
+struct QuadraticRun {
+  kata_dtype_t dtype;
+  QuadraticLaunch a;
+  template <int DK, int DV, int FEAT> kata_status_t operator()() {
+    cudaError_t e = dtype == KATA_DTYPE_F32 ? simt_quadratic<DK, DV, FEAT, float>(a)
+                                            : simt_quadratic<DK, DV, FEAT, __nv_bfloat16>(a);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+  }
+};
+
+struct DecodeRun {
+  kata_dtype_t dtype;
+  DecodeLaunch a;
+  template <int DK, int DV, int FEAT> kata_status_t operator()() {
+    cudaError_t e = dtype == KATA_DTYPE_F32 ? simt_decode<DK, DV, FEAT, float>(a)
+                                            : simt_decode<DK, DV, FEAT, __nv_bfloat16>(a);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+  }
+};
+
+kata_status_t chunked_common(const void *q, const void *k, const void *v, void *o, int B, int H,
+                             int T, int d_k, int d_v, int C, kata_dtype_t dtype,
+                             kata_feature_t feature, float *S_out, float *z_out, void *workspace,
+                             size_t workspace_bytes, kata_stream_t stream_, bool sequential) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || H < 0 || T < 0 || C <= 0) return KATA_ERR_INVALID_ARGUMENT;
+  if (!supported(d_k, d_v, C, dtype, feature)) return KATA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  const int D = (int)kata_state_dim(d_k, feature);
+  if (!workspace) return KATA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return KATA_ERR_WORKSPACE;
+  const int sms = device_sm_count();
+  if (sms <= 0) return KATA_ERR_CUDA;
+  const Split sp = segment_split(BH, T, C, sms, sequential);
+  if (workspace_bytes < workspace_bytes_for(BH, D, d_v, sp)) return KATA_ERR_WORKSPACE;
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  if (BH == 0 || T == 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
+    if (S_out && BH > 0 &&
+        cudaMemsetAsync(S_out, 0, (size_t)BH * D * d_v * sizeof(float), stream) != cudaSuccess)
+      return KATA_ERR_CUDA;
+    if (z_out && BH > 0 &&
+        cudaMemsetAsync(z_out, 0, (size_t)BH * D * sizeof(float), stream) != cudaSuccess)
+      return KATA_ERR_CUDA;
+    return KATA_OK;
+  }
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARGUMENT;
+  unsigned *status = reinterpret_cast<unsigned *>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
+  ChunkedRun run{dtype, ChunkedLaunch{q, k, v, o, BH, T, C, S_out, z_out, status,
+                                      reinterpret_cast<float *>(ws + kHeaderBytes), sp.G,
+                                      sp.seg_len, stream}};
+  return dispatch_shape(d_k, d_v, feature, run);
+}
+
+}  // namespace
+
+extern "C" {
+
+int kata_version(void) { return 100; }
+
+const char *kata_status_string(kata_status_t s) {
+  switch (s) {
+    case KATA_OK: return "KATA_OK";
+    case KATA_ERR_INVALID_ARGUMENT: return "KATA_ERR_INVALID_ARGUMENT";
+    case KATA_ERR_UNSUPPORTED: return "KATA_ERR_UNSUPPORTED";
+    case KATA_ERR_WORKSPACE: return "KATA_ERR_WORKSPACE";
+    case KATA_ERR_CUDA: return "KATA_ERR_CUDA";
+    case KATA_ERR_NONPOSITIVE_NORMALISER: return "KATA_ERR_NONPOSITIVE_NORMALISER";
+  }
+  return "KATA_ERR_UNKNOWN";
+}
+
+size_t kata_state_dim(int d_k, kata_feature_t feature) {
+  if (d_k <= 0) return 0;
+  if (feature == KATA_FEATURE_PSD) return (size_t)d_k * (d_k + 1) / 2;
+  if (feature == KATA_FEATURE_FIRST_ORDER) return (size_t)d_k + 1;
+  return 0;
+}
+
+size_t kata_fwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C,
+                                        kata_dtype_t dtype, kata_feature_t feature) {
+  if (B < 0 || H < 0 || T < 0 || C <= 0) return 0;
+  if (!supported(d_k, d_v, C, dtype, feature)) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return 0;
+  const long long BH = (long long)B * H;
+  const Split sp = segment_split(BH, T, C, sms, false);
+  return workspace_bytes_for(BH, (int)kata_state_dim(d_k, feature), d_v, sp);
+}
+
+kata_status_t kata_fwd_chunked(const void *q, const void *k, const void *v, void *o, int B, int H,
+                               int T, int d_k, int d_v, int C, kata_dtype_t dtype,
+                               kata_feature_t feature, float *S_out, float *z_out,
+                               void *workspace, size_t workspace_bytes, kata_stream_t stream) {
+  return chunked_common(q, k, v, o, B, H, T, d_k, d_v, C, dtype, feature, S_out, z_out, workspace,
+                        workspace_bytes, stream, false);
+}
+
+kata_status_t kata_fwd_chunked_sequential(const void *q, const void *k, const void *v, void *o,
+                                          int B, int H, int T, int d_k, int d_v, int C,
+                                          kata_dtype_t dtype, kata_feature_t feature,
+                                          float *S_out, float *z_out, void *workspace,
+                                          size_t workspace_bytes, kata_stream_t stream) {
+  return chunked_common(q, k, v, o, B, H, T, d_k, d_v, C, dtype, feature, S_out, z_out, workspace,
+                        workspace_bytes, stream, true);
+}
+
+kata_status_t kata_fwd_quadratic(const void *q, const void *k, const void *v, void *o, int B,
+                                 int H, int T, int d_k, int d_v, kata_dtype_t dtype,
+                                 kata_feature_t feature, kata_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || H < 0 || T < 0) return KATA_ERR_INVALID_ARGUMENT;
+  if (!supported(d_k, d_v, 0, dtype, feature)) return KATA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH == 0 || T == 0) return KATA_OK;
+  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARGUMENT;
+  if (BH > 65535) return KATA_ERR_UNSUPPORTED;
+  QuadraticRun run{dtype, QuadraticLaunch{q, k, v, o, BH, T, stream}};
+  return dispatch_shape(d_k, d_v, feature, run);
+}
+
+kata_status_t kata_decode_step(const void *q, const void *k, const void *v, float *S, float *z,
+                               void *y, int B, int H, int d_k, int d_v, kata_dtype_t dtype,
+                               kata_feature_t feature, kata_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || H < 0) return KATA_ERR_INVALID_ARGUMENT;
+  if (!supported(d_k, d_v, 0, dtype, feature)) return KATA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH == 0) return KATA_OK;
+  if (!q || !k || !v || !S || !z || !y) return KATA_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(S) % 16 != 0) return KATA_ERR_INVALID_ARGUMENT;
+  if (BH > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
+  DecodeRun run{dtype, DecodeLaunch{q, k, v, S, z, y, BH, stream}};
+  return dispatch_shape(d_k, d_v, feature, run);
+}
+
+kata_status_t kata_workspace_status(const void *workspace, kata_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!workspace) return KATA_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return KATA_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KATA_ERR_CUDA;
+  if (word & kStatusNonPositiveNormaliser) return KATA_ERR_NONPOSITIVE_NORMALISER;
+  return KATA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// Host-side launch descriptors shared by the C ABI and the kernel files.
+// Each kernel family is instantiated in its own translation unit (one per
+// feature x element type) so that nvcc builds them in parallel.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace kata {
+
+struct ChunkedLaunch {
+  const void *q, *k, *v;
+  void *o;
+  long long BH;
+  int T, C;
+  float *S_out, *z_out;
+  unsigned *status;    // device status word
+  float *agg;          // per-segment increments [BH][G][D][d_v + 1]
+  int G, seg_len;      // segments per head, tokens per segment
+  cudaStream_t stream;
+};
+
+struct QuadraticLaunch {
+  const void *q, *k, *v;
+  void *o;
+  long long BH;
+  int T;
+  cudaStream_t stream;
+};
+
+struct DecodeLaunch {
+  const void *q, *k, *v;
+  float *S, *z;
+  void *y;
+  long long BH;
+  cudaStream_t stream;
+};
+
+template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_chunked(const ChunkedLaunch &a);
+template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_quadratic(const QuadraticLaunch &a);
+template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_decode(const DecodeLaunch &a);
+
+}  // namespace kata
