@@ -144,6 +144,35 @@ KATA_API kata_status_t kata_fwd_chunked_sequential(const void *q, const void *k,
                                           kata_stream_t stream);
 
 /*
+ * kata_fwd_chunked without a caller-provided workspace, for callers that
+ * cannot allocate device memory (for example a host application whose device
+ * memory belongs entirely to another runtime's pool, or latency-critical code
+ * that must not cause the device-wide synchronisation of cudaMalloc /
+ * cudaFree). The paper has no counterpart: this is a library convenience.
+ *
+ * Scratch is one fixed device array of KATA_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * inside the library, held by every GPU that loads it until the process
+ * exits. Same arguments and results as kata_fwd_chunked minus the workspace.
+ *  - Returns KATA_ERR_WORKSPACE, before launching anything, when the problem
+ *    needs more scratch than the array holds, i.e. when
+ *    kata_fwd_chunked_workspace_bytes(...) > KATA_NOALLOC_SCRATCH_BYTES.
+ *  - The first call on a device looks up the array's device address for that
+ *    device (cudaGetSymbolAddress with the device current); make that first
+ *    call before any stream capture.
+ *  - All calls share the array, which keeps the last call's contents (each
+ *    call clears the status word it needs to start at zero). Calls whose work
+ *    overlaps on the GPU (different streams, different host threads) race on
+ *    it: serialise them.
+ *  - The device status word is not readable from outside; rows with a
+ *    non-positive normaliser give non-finite outputs as usual.
+ */
+#define KATA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+KATA_API kata_status_t kata_fwd_chunked_noalloc(const void *q, const void *k, const void *v,
+                                                void *o, int B, int H, int T, int d_k, int d_v,
+                                                int C, kata_dtype_t dtype, kata_feature_t feature,
+                                                float *S_out, float *z_out, kata_stream_t stream);
+
+/*
  * Flash-attention-style quadratic causal forward (explainer 2.3, operating
  * point 1: O(T^2), no state is materialised). For each query block the key
  * blocks up to the diagonal are visited; P = (Q K^T)^2 (or 1 + Q K^T) masked,
