@@ -26,6 +26,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+W_DECODE_BATCH = 256
 METRIC = "KATA causal fwd tokens/sec at T=131072 (chunked) and % of tensor/HBM roofline"
 UNIT = "tokens/s"
 NOMINAL_FP32_TFLOPS_PER_SM_GHZ = 128 * 2 / 1000.0   # 128 FP32 lanes x FMA, per GHz, in TFLOP/s
@@ -34,6 +35,7 @@ NOMINAL_FP32_TFLOPS_PER_SM_GHZ = 128 * 2 / 1000.0   # 128 FP32 lanes x FMA, per 
 #   tensor: bf16 tensor-core contraction;  alu: fp32 FFMA on the CUDA cores;
 #   hbm: streaming kernel.
 KERNEL_BOUND = {
+    "tc_quadratic": "tensor",
     "simt_segment_pass": "alu",
     "simt_segment_increment": "alu",
     "simt_quadratic": "alu",
@@ -237,20 +239,60 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     kbuild.build()
-    w = W.WORKLOADS[args.workload]
-    if args.T:
-        w = w.with_T(args.T)
     dev = torch.device("cuda", local_rank)
-    # seeded synthetic inputs, generated on the device (one batch per rank)
+    form = args.form
+    w = W.WORKLOADS[args.workload if form != "first_order" else "first_order64k_bf16"]
+    if form == "quadratic":
+        w = w.with_T(args.T or W.LONG_QUADRATIC_T)
+    elif args.T:
+        w = w.with_T(args.T)
     from dataclasses import replace
-    w_rank = replace(w, seed=w.seed + 1000 * rank)
-    q, k, v = W.make_inputs(w_rank, device=dev)
-    o = torch.empty_like(v)
-    ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
+    w = replace(w, seed=w.seed + 1000 * rank)     # one seeded batch per rank
     stream = torch.cuda.current_stream()
+    if form == "decode":
+        B, H = args.decode_batch, W.DECODE_HEADS
+        q, k, v = W.make_decode_inputs(B, H, device=dev)
+        # prior state per sequence: 4096 seeded tokens accumulated by the library
+        kp, vp = W.make_decode_prior_tokens(B, H, device=dev)
+        _, S, z = api.fwd_chunked(kp, kp, vp, 128, "psd", return_state=True)
+        del kp, vp
+        o = torch.empty_like(v)
+        ws = None
 
-    def step():
-        api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws)
+        def step():
+            api.kata_decode_step(q, k, v, S, z, o)
+        tokens_per_step = B
+        token_heads = B * H
+        D = api.state_dim(W.DECODE_DK)
+        flops_th = 2 * D * W.DECODE_DV * 2 + 3 * D
+        bytes_th = 2 * 4 * D * (W.DECODE_DV + 1) + 2 * (2 * W.DECODE_DK + 2 * W.DECODE_DV)
+        config = {"workload": f"decode_b{B}_h{H}", "B": B, "H": H, "d_k": W.DECODE_DK,
+                  "d_v": W.DECODE_DV, "feature": "psd", "form": "decode step",
+                  "l2": "state larger than L2 (no flush needed)"}
+    else:
+        q, k, v = W.make_inputs(w, device=dev)
+        o = torch.empty_like(v)
+        if form == "quadratic":
+            ws = None
+
+            def step():
+                api.kata_fwd_quadratic(q, k, v, o, w.feature)
+            flops_th = (w.T + 1) / 2 * (2 * w.d_k + 2 * w.d_v + 2)
+            _, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
+        else:
+            ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
+            seq = form == "sequential"
+
+            def step():
+                api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws, sequential=seq)
+            flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
+        tokens_per_step = w.B * w.T
+        token_heads = w.B * w.H * w.T
+        config = workload_config(w)
+        config["form"] = {"chunked": "chunked (segmented scan carry)",
+                          "sequential": "chunked (sequential carry)",
+                          "first_order": "chunked first-order (segmented scan carry)",
+                          "quadratic": "quadratic (flash-style)"}[form]
 
     def barrier():
         if world > 1:
@@ -259,9 +301,10 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    st = api.kata_workspace_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {st} after warm-up")
+    if ws is not None:
+        st = api.kata_workspace_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status {st} after warm-up")
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clocks:
@@ -281,7 +324,6 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    tokens_per_step = w.B * w.T
     value = world * tokens_per_step / (ms / 1e3)
 
     # roofline of the dominant kernel, timed live by the library's events
@@ -289,8 +331,6 @@ def run_ours(args, rank, world, local_rank):
     dom = max(prof, key=lambda n: prof[n][1])
     launches, dom_ms = prof[dom]
     dom_avg_s = dom_ms / launches / 1e3
-    flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
-    token_heads = w.B * w.H * w.T
     # achieved = the step's algorithmic work / one launch of the dominant kernel
     per_launch_units = token_heads
     bound = KERNEL_BOUND.get(dom, "tensor")
@@ -320,7 +360,7 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and form != "decode":
         qh = q.cpu().pin_memory()
         kh = k.cpu().pin_memory()
         vh = v.cpu().pin_memory()
@@ -330,7 +370,7 @@ def run_ours(args, rank, world, local_rank):
             q.copy_(qh, non_blocking=True)
             k.copy_(kh, non_blocking=True)
             v.copy_(vh, non_blocking=True)
-            api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws)
+            step()
             oh.copy_(o, non_blocking=True)
 
         for _ in range(2):
@@ -354,7 +394,7 @@ def run_ours(args, rank, world, local_rank):
                "d2h_bytes_per_step": o.numel() * o.element_size(), "ms_per_step": ms_e2e}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and form == "chunked":
         val, sample = oracle_sample(W.WORKLOADS[args.workload], budget_s=args.cpu_budget)
         cpu = {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": sample}
@@ -364,10 +404,10 @@ def run_ours(args, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(w) | {"parallelism": f"replicas x{world}"},
+            "config": config | {"parallelism": f"replicas x{world}"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
             "kernels": {n: {"launches": c, "avg_ms": t / c} for n, (c, t) in prof.items()},
-            "clocks": clocks.summary(), "token_heads_per_s": value * w.H,
+            "clocks": clocks.summary(), "token_heads_per_s": value * token_heads / tokens_per_step,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -380,6 +420,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long131k_bf16")
+    ap.add_argument("--form", default="chunked",
+                    choices=["chunked", "sequential", "first_order", "quadratic", "decode"],
+                    help="chunked is the headline; the others are secondary measurements")
+    ap.add_argument("--decode-batch", type=int, default=W_DECODE_BATCH)
     ap.add_argument("--T", type=int, default=0, help="override T (profiling a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

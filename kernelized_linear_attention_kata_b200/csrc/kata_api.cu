@@ -96,8 +96,11 @@ struct QuadraticRun {
   kata_dtype_t dtype;
   QuadraticLaunch a;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
-    cudaError_t e = dtype == KATA_DTYPE_F32 ? simt_quadratic<DK, DV, FEAT, float>(a)
-                                            : simt_quadratic<DK, DV, FEAT, __nv_bfloat16>(a);
+    cudaError_t e = cudaErrorNotSupported;
+    if (dtype == KATA_DTYPE_BF16) e = tc_quadratic(a, DK, DV, FEAT);
+    if (e == cudaErrorNotSupported)
+      e = dtype == KATA_DTYPE_F32 ? simt_quadratic<DK, DV, FEAT, float>(a)
+                                  : simt_quadratic<DK, DV, FEAT, __nv_bfloat16>(a);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
   }
 };

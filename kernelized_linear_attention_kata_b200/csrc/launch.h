@@ -36,6 +36,11 @@ struct DecodeLaunch {
   cudaStream_t stream;
 };
 
+// Tensor-core kernels (bf16 only). They return cudaErrorNotSupported, having
+// launched nothing, for shapes or alignments they do not handle; the caller
+// then runs the CUDA-core kernel instead.
+cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature);
+
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_chunked(const ChunkedLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_quadratic(const QuadraticLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_decode(const DecodeLaunch &a);
