@@ -73,7 +73,10 @@ typedef enum {
     KATA_ERR_UNSUPPORTED = 2,      /* shape / dtype / feature not built      */
     KATA_ERR_WORKSPACE = 3,        /* workspace missing, too small, unaligned */
     KATA_ERR_CUDA = 4,             /* a CUDA call or launch failed           */
-    KATA_ERR_NONPOSITIVE_NORMALISER = 5 /* device: some row had den <= 0     */
+    KATA_ERR_NONPOSITIVE_NORMALISER = 5, /* device: some row had den <= 0    */
+    KATA_ERR_DEVICE_TIMEOUT = 6    /* device: a bounded wait inside a kernel
+                                      gave up (a library defect); outputs of
+                                      that call are undefined               */
 } kata_status_t;
 
 typedef enum { KATA_DTYPE_F32 = 0, KATA_DTYPE_BF16 = 1 } kata_dtype_t;

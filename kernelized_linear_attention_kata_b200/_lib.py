@@ -20,6 +20,7 @@ KATA_ERR_UNSUPPORTED = 2
 KATA_ERR_WORKSPACE = 3
 KATA_ERR_CUDA = 4
 KATA_ERR_NONPOSITIVE_NORMALISER = 5
+KATA_ERR_DEVICE_TIMEOUT = 6
 
 KATA_DTYPE_F32 = 0
 KATA_DTYPE_BF16 = 1

@@ -11,7 +11,7 @@ namespace kata {
 enum Feature : int { kPSD = 0, kFirstOrder = 1 };
 
 // Status bits written by kernels into the first word of the workspace.
-enum : unsigned { kStatusNonPositiveNormaliser = 1u };
+enum : unsigned { kStatusNonPositiveNormaliser = 1u, kStatusDeviceTimeout = 2u };
 
 __host__ __device__ constexpr int state_dim(int d_k, int feat) {
   return feat == kPSD ? d_k * (d_k + 1) / 2 : d_k + 1;

@@ -55,8 +55,17 @@ Split segment_split(long long BH, int T, int C, int sms, bool sequential) {
   return {Gr, per * C};
 }
 
-size_t workspace_bytes_for(long long BH, int D, int d_v, const Split &sp) {
-  const size_t agg = (size_t)BH * (size_t)sp.G * (size_t)D * (size_t)(d_v + 1) * sizeof(float);
+// Floats of one segment increment: the CUDA-core kernels keep [D][d_v + 1]
+// (z as the last column), the tensor-core kernel keeps [D][d_v] then the
+// d_k x d_k matrix sum k k^T; the workspace holds the larger.
+size_t increment_floats(int D, int d_k, int d_v) {
+  const size_t simt = (size_t)D * (size_t)(d_v + 1);
+  const size_t tc = (size_t)D * (size_t)d_v + (size_t)d_k * (size_t)d_k;
+  return simt > tc ? simt : tc;
+}
+
+size_t workspace_bytes_for(long long BH, int D, int d_k, int d_v, const Split &sp) {
+  const size_t agg = (size_t)BH * (size_t)sp.G * increment_floats(D, d_k, d_v) * sizeof(float);
   return kHeaderBytes + align_up(agg, kAlign);
 }
 
@@ -86,8 +95,11 @@ struct ChunkedRun {
   kata_dtype_t dtype;
   ChunkedLaunch a;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
-    cudaError_t e = dtype == KATA_DTYPE_F32 ? simt_chunked<DK, DV, FEAT, float>(a)
-                                            : simt_chunked<DK, DV, FEAT, __nv_bfloat16>(a);
+    cudaError_t e = cudaErrorNotSupported;
+    if (dtype == KATA_DTYPE_BF16 && tc_chunked_supported(a, DK, DV, a.C, FEAT)) e = tc_chunked(a);
+    if (e == cudaErrorNotSupported)
+      e = dtype == KATA_DTYPE_F32 ? simt_chunked<DK, DV, FEAT, float>(a)
+                                  : simt_chunked<DK, DV, FEAT, __nv_bfloat16>(a);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
   }
 };
@@ -129,7 +141,7 @@ kata_status_t chunked_common(const void *q, const void *k, const void *v, void *
   const int sms = device_sm_count();
   if (sms <= 0) return KATA_ERR_CUDA;
   const Split sp = segment_split(BH, T, C, sms, sequential);
-  if (workspace_bytes < workspace_bytes_for(BH, D, d_v, sp)) return KATA_ERR_WORKSPACE;
+  if (workspace_bytes < workspace_bytes_for(BH, D, d_k, d_v, sp)) return KATA_ERR_WORKSPACE;
   unsigned char *ws = static_cast<unsigned char *>(workspace);
   if (BH == 0 || T == 0) {
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
@@ -164,6 +176,7 @@ const char *kata_status_string(kata_status_t s) {
     case KATA_ERR_WORKSPACE: return "KATA_ERR_WORKSPACE";
     case KATA_ERR_CUDA: return "KATA_ERR_CUDA";
     case KATA_ERR_NONPOSITIVE_NORMALISER: return "KATA_ERR_NONPOSITIVE_NORMALISER";
+    case KATA_ERR_DEVICE_TIMEOUT: return "KATA_ERR_DEVICE_TIMEOUT";
   }
   return "KATA_ERR_UNKNOWN";
 }
@@ -183,7 +196,7 @@ size_t kata_fwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, i
   if (sms <= 0) return 0;
   const long long BH = (long long)B * H;
   const Split sp = segment_split(BH, T, C, sms, false);
-  return workspace_bytes_for(BH, (int)kata_state_dim(d_k, feature), d_v, sp);
+  return workspace_bytes_for(BH, (int)kata_state_dim(d_k, feature), d_k, d_v, sp);
 }
 
 kata_status_t kata_fwd_chunked(const void *q, const void *k, const void *v, void *o, int B, int H,
@@ -239,6 +252,7 @@ kata_status_t kata_workspace_status(const void *workspace, kata_stream_t stream_
   unsigned word = 0;
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
     return KATA_ERR_CUDA;
+  if (word & kStatusDeviceTimeout) return KATA_ERR_DEVICE_TIMEOUT;
   if (word & kStatusNonPositiveNormaliser) return KATA_ERR_NONPOSITIVE_NORMALISER;
   return KATA_OK;
 }

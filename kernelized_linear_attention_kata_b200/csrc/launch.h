@@ -40,6 +40,9 @@ struct DecodeLaunch {
 // launched nothing, for shapes or alignments they do not handle; the caller
 // then runs the CUDA-core kernel instead.
 cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature);
+bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
+cudaError_t tc_chunked(const ChunkedLaunch &a);
+size_t tc_chunked_agg_floats();   // floats of one segment increment
 
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_chunked(const ChunkedLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_quadratic(const QuadraticLaunch &a);

@@ -284,3 +284,47 @@ def test_unsupported_shape_raises():
     v = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises((KataError, ValueError)):
         api.fwd_chunked(q, q, v, 64)
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core chunked path (bf16, PSD, d_k = 32, d_v = 64, C = 128)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,H,T", [(1, 1, 1), (1, 2, 127), (1, 3, 128), (2, 2, 129), (1, 4, 1000),
+                                   (1, 2, 5000), (2, 80, 300)])
+def test_tc_chunked_c128_shapes_and_state(B, H, T):
+    w = W.Workload("tc", B=B, H=H, T=T, d_k=32, d_v=64, C=128, dtype="bf16", feature="psd",
+                   seed=1000 + T + H, recipe="unit")
+    q, k, v = W.make_inputs(w)
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    ref = np.empty((B, H, T, 64))
+    S_ref = np.empty((B, H, 528, 64))
+    z_ref = np.empty((B, H, 528))
+    for b in range(B):
+        for h in range(H):
+            ref[b, h], S_ref[b, h], z_ref[b, h] = O.forward_chunked(qn[b, h], kn[b, h], vn[b, h], 128,
+                                                                    return_state=True)
+    qd, kd, vd = dev(q, k, v)
+    for seq in (False, True):
+        y, S, z = api.fwd_chunked(qd, kd, vd, 128, "psd", return_state=True, sequential=seq)
+        e = rel_err(y.float().cpu().numpy(), ref)
+        assert e <= TOL["bf16"], (seq, e)
+        # the update MMA takes the feature products k_i k_j in bf16 (relative
+        # rounding 2^-9 per term); the state is held to 1e-2 of its largest
+        # entry. z comes from K^T K with exact fp32 products.
+        assert np.max(np.abs(S.cpu().numpy() - S_ref)) <= 1e-2 * np.abs(S_ref).max(), seq
+        assert np.max(np.abs(z.cpu().numpy() - z_ref)) <= 1e-4 * np.abs(z_ref).max(), seq
+
+
+def test_tc_chunked_reports_nonpositive_normaliser():
+    w = W.Workload("tcz", B=1, H=2, T=600, d_k=32, d_v=64, C=128, dtype="bf16", feature="psd",
+                   seed=8, recipe="unit")
+    q, k, v = dev(*W.make_inputs(w))
+    ws = api.alloc_workspace(1, 2, 600, 32, 64, 128)
+    o = torch.empty_like(v)
+    api.kata_fwd_chunked(q, k, v, o, 128, "psd", workspace=ws)
+    assert api.kata_workspace_status(ws) == KATA_OK
+    q2 = q.clone()
+    q2[0, 0, 300] = 0
+    api.kata_fwd_chunked(q2, k, v, o, 128, "psd", workspace=ws)
+    assert api.kata_workspace_status(ws) == KATA_ERR_NONPOSITIVE_NORMALISER

@@ -58,7 +58,7 @@ def test_state_dim(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert lib.kata_status_string(code).decode().startswith("KATA_")
     assert lib.kata_status_string(99) == b"KATA_ERR_UNKNOWN"
     assert lib.kata_version() >= 100
