@@ -24,19 +24,25 @@
 // state is converted to the library's row-major (i <= j) order only where it
 // leaves the kernel (S_out, z_out).
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocation and
-// MMA issue (one lane), warps 2-5 math: thread r owns TMEM lane r, which is
-// token r of the chunk for the token-major tiles and feature row r of each
-// 128-feature state tile.
+// Warp roles (352 threads): warp 0 TMA producer; warp 1 TMEM allocation and
+// the query-side MMAs (Q K^T, P V, U, the readout into O); warp 10 the
+// state-side MMAs (the update of S and Z) - two issuing threads so that one's
+// waits are covered by the other's MMAs; warps 2-5, the query side: the
+// intra-chunk P, the query features into the ring, the epilogue; warps 6-9,
+// the key side: the key features into the ring, the bf16 snapshot of the
+// state after each update, the carry-in and the state written out. Math
+// thread r owns TMEM lane r (quarter = warp mod 4): token r of the chunk for
+// the token-major tiles, feature row r of each 128-feature state tile.
 //
 // Tensor memory (512 columns, fp32):
 //   [  0, 320)  S, five 128-feature tiles of 64 columns (tile 4: 16 rows used)
 //   [320, 352)  Z (lanes 0..31)
 //   [352, 384)  U = Q_c Z_c (den of the inter-chunk part)
 //   [384, 512)  Q_c K_c^T; then P (bf16, in place, [384, 448)) and O ([448, 512))
-// Shared memory: two TMA stages of (Q, K, V) tiles, the bf16 snapshot of S_c
-// (the readout's B operand) and of Z_c, and a two-slot ring of 128-feature
-// phi tiles (the readout's A operand for Q, the update's A operand for K).
+// Shared memory (220 KB): the Q tile (single buffer), two TMA stages of K and
+// V, the bf16 snapshot of S_c (the readout's B operand) and of Z_c, and a
+// ring of three 128-feature slots shared by the query features (readout A
+// operand) and the key features (update A operand).
 #include "common.cuh"
 #include "launch.h"
 #include "profile.h"
@@ -52,31 +58,52 @@ constexpr int kC = 128;            // chunk
 constexpr int kDK = 32;
 constexpr int kDV = 64;
 constexpr int kD = 528;
-constexpr int kTiles = 5;          // ceil(528 / 128)
-constexpr int kThreads = 192;
+constexpr int kTiles = 5;          // 128-feature state tiles: ceil(528 / 128)
+constexpr int kThreads = 352;      // 11 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColZ = 320, kColU = 352, kColX = 384, kColO = 448;
 constexpr int kAggFloats = kD * kDV + kDK * kDK;      // one segment increment
 
-// Shared memory layout (bytes from a 1024-aligned base).
-constexpr int kStageBytes = 32768;                    // Q 8 KB | K 8 KB | V 16 KB
-constexpr int kOffQ = 0, kOffK = 8192, kOffV = 16384;
-constexpr int kOffStages = 0;
-constexpr int kOffSnap = 2 * kStageBytes;             // S_c bf16 [528][64], 128 B rows
-constexpr int kSnapBytes = kD * 128;
-constexpr int kOffZSnap = kOffSnap + kSnapBytes;      // Z_c bf16 [32][32], 64 B rows
-constexpr int kOffSlots = kOffZSnap + 2048;           // two 32 KB phi slots
-constexpr int kSlotBytes = 32768;
-constexpr int kOffBars = kOffSlots + 2 * kSlotBytes;
-enum {
-  kBarKvFull = 0, kBarKvEmpty = 2, kBarSFull = 4, kBarPFull, kBarOFull, kBarUpdFull, kBarXFree,
-  kBarSnapFull, kBarSlotFull = 10, kBarSlotEmpty = 12, kNumBars = 14
+// Shared memory layout (bytes from a 1024-aligned base). Features travel
+// through two rings, each with one producer set and one consumer warp (an
+// mbarrier parity wait is only unambiguous for a single consumer in order):
+//   query ring: 16 KB slots of 128 token rows x 64 query features (readout
+//               A operand, K-major), nine uses per chunk;
+//   key ring:   32 KB slots of 128 token rows x 128 key features, as two
+//               64-feature groups 16 KB apart (update A operand, MN-major),
+//               five uses per chunk, one per state tile.
+//   forward pass:  Q 8 KB | K 2 x 8 KB | V 2 x 16 KB | S_c bf16 66 KB |
+//                  Z_c bf16 2 KB | query ring 2 x 16 KB | key ring 2 x 32 KB
+//   increments:    K 2 x 8 KB | V 2 x 16 KB | key ring 5 x 32 KB
+constexpr int kQSlotBytes = 16384;
+constexpr int kKSlotBytes = 32768;
+constexpr int kQSlots = 9;          // 64-feature readout slots per chunk
+template <bool AGG>
+struct Layout {
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = AGG ? 0 : 8192;
+  static constexpr int kOffV = kOffK + 16384;
+  static constexpr int kOffSnap = kOffV + 32768;      // [528][64] bf16, 128 B rows (pass only)
+  static constexpr int kOffZSnap = kOffSnap + (AGG ? 0 : kD * 128);
+  static constexpr int kOffQRing = kOffZSnap + (AGG ? 0 : 2048);
+  static constexpr int kQRingSlots = AGG ? 0 : 2;
+  static constexpr int kOffKRing = kOffQRing + kQRingSlots * kQSlotBytes;
+  static constexpr int kKRingSlots = AGG ? 5 : 2;
+  static constexpr int kOffBars = kOffKRing + kKRingSlots * kKSlotBytes;
+  static constexpr int kSmemBytes = kOffBars + 1024 + 1024;   // barriers + alignment slack
+  static_assert(kOffV % 1024 == 0 && kOffSnap % 1024 == 0 && kOffZSnap % 1024 == 0 &&
+                kOffQRing % 1024 == 0 && kOffKRing % 1024 == 0,
+                "swizzle atoms need 1024-byte alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
-constexpr int kOffTmemSlot = kOffBars + 8 * kNumBars;
-constexpr int kOffAbort = kOffTmemSlot + 4;
-constexpr int kSmemBytes = kOffAbort + 4 + 1024;      // + alignment slack
-static_assert(kOffSnap % 1024 == 0 && kOffZSnap % 1024 == 0 && kOffSlots % 1024 == 0, "align");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
+enum {
+  kBarQFull = 0, kBarQEmpty, kBarKvFull, kBarKvEmpty = kBarKvFull + 2, kBarSFull = kBarKvEmpty + 2,
+  kBarPFull, kBarOFull, kBarXFree, kBarUpdFull, kBarZDone, kBarZSnap, kBarTileDone,
+  kBarTileSnap = kBarTileDone + 5, kBarQRingFull = kBarTileSnap + 5, kBarQRingEmpty = kBarQRingFull + 2,
+  kBarKRingFull = kBarQRingEmpty + 2, kBarKRingEmpty = kBarKRingFull + 5, kNumBars = kBarKRingEmpty + 5
+};
+constexpr int kBarBytes = 8 * kNumBars;
+static_assert(kBarBytes + 8 <= 1024, "barrier area");
 
 // Byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-row tile
 // with the 128-byte swizzle (atoms of 8 rows x 128 B).
@@ -109,32 +136,48 @@ __device__ __forceinline__ int abi_row(int f) {
   return i * kDK - i * (i - 1) / 2 + (j - i);
 }
 
-// Writes the phi tile of slot s (features 128 s .. 128 s + 127) for one token
-// row into a 32 KB slot (two 64-feature groups of 128-byte rows). P[l] holds
-// the bf16 pair (x_l, x_(l+1) mod 32); M[l] is the multiplier pair for the
-// partner index (x doubled off the diagonal on the query side).
+// One 16-byte chunk (8 features (d, l0 .. l0+7)) of a token's feature row.
+// P[l] holds the bf16 pair (x_l, x_(l+1) mod 32); M is P, or P doubled for
+// the query's off-diagonal multiplicity.
+__device__ __forceinline__ uint4 phi_chunk(int d, int l0, const uint32_t (&P)[32],
+                                           const uint32_t (&M)[32]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int l = l0 + 2 * k;
+    w[k] = bmul2(P[l], M[(l + d) & 31]);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Query features of readout slot s (features 64 s .. 64 s + 63, offsets
+// d = 2 s, 2 s + 1; slot 8 holds only (16, l < 16)) for one token row, with
+// the off-diagonal multiplicity 2 (P2 = 2 P).
+__device__ __forceinline__ void write_q_slot(uint8_t *slot, int row, int s, const uint32_t (&P)[32],
+                                             const uint32_t (&P2)[32]) {
+#pragma unroll
+  for (int cc = 0; cc < 8; ++cc) {
+    if (s == 8 && cc >= 2) continue;
+    const int d = 2 * s + (cc >> 2);
+    const uint4 v = d == 0 ? phi_chunk(d, (cc & 3) * 8, P, P) : phi_chunk(d, (cc & 3) * 8, P, P2);
+    *reinterpret_cast<uint4 *>(slot + sw128(row, cc)) = v;
+  }
+}
+
+// Features of state tile m (128 m .. 128 m + 127; two 64-feature groups 16
+// KB apart; tile 4 holds only (16, l < 16)) for one token row. QUERY doubles
+// the off-diagonal features (the readout side).
 template <bool QUERY>
-__device__ __forceinline__ void write_phi_slot(uint8_t *slot, int row, int s, const uint32_t (&P)[32],
-                                               const uint32_t (&P2)[32]) {
+__device__ __forceinline__ void write_tile(uint8_t *slot, int row, int m, const uint32_t (&P)[32],
+                                           const uint32_t (&P2)[32]) {
 #pragma unroll
   for (int g2 = 0; g2 < 2; ++g2) {
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
-      const int d = 4 * s + 2 * g2 + (cc >> 2);
-      const int l0 = (cc & 3) * 8;
-      if (s == 4 && (g2 != 0 || cc >= 2)) continue;         // only (16, l < 16) in slot 4
-      uint4 v;
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int l = l0 + 2 * k;
-        const int m = (l + d) & 31;
-        w[k] = bmul2(P[l], (QUERY && d != 0) ? P2[m] : P[m]);
-      }
-      v.x = w[0];
-      v.y = w[1];
-      v.z = w[2];
-      v.w = w[3];
+      if (m == 4 && (g2 != 0 || cc >= 2)) continue;
+      const int d = 4 * m + 2 * g2 + (cc >> 2);
+      const uint4 v = (QUERY && d != 0) ? phi_chunk(d, (cc & 3) * 8, P, P2)
+                                        : phi_chunk(d, (cc & 3) * 8, P, P);
       *reinterpret_cast<uint4 *>(slot + g2 * 16384 + sw128(row, cc)) = v;
     }
   }
@@ -158,18 +201,35 @@ __device__ __forceinline__ void load_pairs(const uint8_t *tile, int row, uint32_
   }
 }
 
+__device__ __forceinline__ uint4 pack8(const uint32_t *a) {
+  return make_uint4(tc::pack_bf16x2(__uint_as_float(a[0]), __uint_as_float(a[1])),
+                    tc::pack_bf16x2(__uint_as_float(a[2]), __uint_as_float(a[3])),
+                    tc::pack_bf16x2(__uint_as_float(a[4]), __uint_as_float(a[5])),
+                    tc::pack_bf16x2(__uint_as_float(a[6]), __uint_as_float(a[7])));
+}
+
+// Math-set synchronisation: every thread of the set waits and arrives
+// (counted per thread), so no lane depends on another lane's wait.
+constexpr uint32_t kSetArrivals = 128;
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) { mbar_arrive(bar); }
+
 template <bool AGG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, __nv_bfloat16 *__restrict__ o,
                   float *__restrict__ agg, float *__restrict__ S_out, float *__restrict__ z_out,
                   unsigned *__restrict__ status, int T, int G_grid, int G_total, int seg_len) {
+  using L = Layout<AGG>;
+  constexpr int NK = L::kKRingSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBars);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffBars + kBarBytes);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffBars + kBarBytes + 4);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -180,18 +240,36 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   const int nchunks = (t1 - t0 + kC - 1) / kC;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[kBarKvFull + s], 1);
-      mbar_init(&bars[kBarKvEmpty + s], 1 + 128);
-      mbar_init(&bars[kBarSlotFull + s], 128);
-      mbar_init(&bars[kBarSlotEmpty + s], 1);
+    // arrival counts: 1 for a TMA transaction or an MMA commit,
+    // kSetArrivals for the threads of a math set
+    constexpr uint32_t A = kSetArrivals;
+    mbar_init(&bars[kBarQFull], 1);
+    mbar_init(&bars[kBarQEmpty], 1 + A);
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(&bars[kBarKvFull + st], 1);
+      mbar_init(&bars[kBarKvEmpty + st], (AGG ? 1 : 2) + A);   // MMA warp(s) + key side
     }
     mbar_init(&bars[kBarSFull], 1);
-    mbar_init(&bars[kBarPFull], 128);
+    mbar_init(&bars[kBarPFull], A);
     mbar_init(&bars[kBarOFull], 1);
+    mbar_init(&bars[kBarXFree], A);
     mbar_init(&bars[kBarUpdFull], 1);
-    mbar_init(&bars[kBarXFree], 128);
-    mbar_init(&bars[kBarSnapFull], 128);
+    // done-barriers of the snapshots: one commit from each issuing warp (the
+    // readout / U that read the old snapshot, the update that wrote the new state)
+    mbar_init(&bars[kBarZDone], 2);
+    mbar_init(&bars[kBarZSnap], A);
+    for (int m = 0; m < 5; ++m) {
+      mbar_init(&bars[kBarTileDone + m], 2);
+      mbar_init(&bars[kBarTileSnap + m], A);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&bars[kBarQRingFull + k], A);
+      mbar_init(&bars[kBarQRingEmpty + k], 1);
+    }
+    for (int k = 0; k < NK; ++k) {
+      mbar_init(&bars[kBarKRingFull + k], A);
+      mbar_init(&bars[kBarKRingEmpty + k], 1);
+    }
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -203,6 +281,18 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  uint8_t *qring = smem + L::kOffQRing;
+  uint8_t *kring = smem + L::kOffKRing;
+
+  // Producer side of a ring (one math warp set): use u of a ring with n
+  // slots may be written once its previous occupant (use u - n) is consumed.
+  auto ring_acquire = [&](uint64_t *empty, int n, int u) -> bool {
+    return u < n || warp_wait(&empty[u % n], ((u / n) - 1) & 1, abort_flag);
+  };
+  auto ring_publish = [&](uint64_t *full, int n, int u) {
+    fence_async_smem();
+    warp_arrive(&full[u % n]);
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA
@@ -210,20 +300,26 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       tma_prefetch_desc(&tmk);
       tma_prefetch_desc(&tmv);
       if (!AGG) tma_prefetch_desc(&tmq);
-      const uint32_t bytes = AGG ? 8192 + 16384 : 8192 * 2 + 16384;
       for (int i = 0; i < nchunks; ++i) {
         const int st = i & 1;
-        if (i >= 2 && !mbar_wait(&bars[kBarKvEmpty + st], ((i >> 1) - 1) & 1, abort_flag)) break;
-        uint8_t *stage = smem + kOffStages + st * kStageBytes;
         const int row = t0 + i * kC;
-        mbar_arrive_expect_tx(&bars[kBarKvFull + st], bytes);
-        if (!AGG) tma_load_3d(stage + kOffQ, &tmq, &bars[kBarKvFull + st], 0, row, bh);
-        tma_load_3d(stage + kOffK, &tmk, &bars[kBarKvFull + st], 0, row, bh);
-        tma_load_3d(stage + kOffV, &tmv, &bars[kBarKvFull + st], 0, row, bh);
+        if (!AGG) {
+          if (i >= 1 && !mbar_wait(&bars[kBarQEmpty], (i - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&bars[kBarQFull], 8192);
+          tma_load_3d(smem + L::kOffQ, &tmq, &bars[kBarQFull], 0, row, bh);
+        }
+        if (i >= 2 && !mbar_wait(&bars[kBarKvEmpty + st], ((i >> 1) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&bars[kBarKvFull + st], 8192 + 16384);
+        tma_load_3d(smem + L::kOffK + 8192 * st, &tmk, &bars[kBarKvFull + st], 0, row, bh);
+        tma_load_3d(smem + L::kOffV + 16384 * st, &tmv, &bars[kBarKvFull + st], 0, row, bh);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 10) {
     // ------------------------------------------------------------ MMA issue
+    // Two issuing warps with independent accumulators, so that one's waits
+    // are covered by the other's MMAs: warp 1 issues the query side (Q K^T,
+    // P V, U, the readout into O); warp 10 issues the state side (the update
+    // of S and Z).
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t id_pv = idesc_bf16(128, kDV, false, true);
@@ -231,86 +327,217 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       constexpr uint32_t id_ro = idesc_bf16(128, kDV, false, true);
       constexpr uint32_t id_up = idesc_bf16(128, kDV, true, true);
       constexpr uint32_t id_z = idesc_bf16(128, 32, true, true);
-      const uint32_t snap = smem_u32(smem + kOffSnap);
-      const uint32_t zsnap = smem_u32(smem + kOffZSnap);
-      const uint32_t slots = smem_u32(smem + kOffSlots);
-      int u = 0;                                   // slot uses so far
+      const uint32_t qa = smem_u32(smem + L::kOffQ);
+      const uint32_t qring_a = smem_u32(qring), kring_a = smem_u32(kring);
+      // Descriptors are built once; operands at other offsets of the same
+      // layout differ only in the start-address field (bytes / 16).
+      auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+      const uint64_t d_q = smem_desc(qa, 16, 512, kSw64);                       // Q, K-major
+      const uint64_t d_z = smem_desc(smem_u32(smem + L::kOffZSnap), 16, 512, kSw64);
+      const uint64_t d_snap = smem_desc(smem_u32(smem + L::kOffSnap), 16384, 1024, kSw128);
+      const uint64_t d_qring = smem_desc(qring_a, 16, 1024, kSw128);            // readout A
+      const uint64_t d_kring = smem_desc(kring_a, 16384, 1024, kSw128);         // update A
+      const uint64_t d_k_k = smem_desc(smem_u32(smem + L::kOffK), 16, 512, kSw64);     // K, K-major
+      const uint64_t d_k_mn = smem_desc(smem_u32(smem + L::kOffK), 8192, 512, kSw64);  // K, MN-major
+      const uint64_t d_v = smem_desc(smem_u32(smem + L::kOffV), 16384, 1024, kSw128);  // V, MN-major
+      // Ring slots are shared memory written by threads (ordered for the
+      // tensor core by their proxy fence and the mbarrier), so ring waits
+      // need no tcgen05 fence; only hand-offs of tensor memory do.
+      // Two barriers tested back to back so that their latencies overlap.
+      auto wait2 = [&](uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2) -> bool {
+        const bool a = mbar_test_wait(b1, p1), b = mbar_test_wait(b2, p2);
+        if (a && b) return true;
+        return (a || mbar_wait(b1, p1, abort_flag)) && (b || mbar_wait(b2, p2, abort_flag));
+      };
       bool ok = true;
-      for (int i = 0; ok && i < nchunks; ++i) {
-        const int st = i & 1;
-        const uint32_t stage = smem_u32(smem + kOffStages + st * kStageBytes);
-        if (!(ok = mbar_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
-        if (!AGG) {
-          if (i > 0 && !(ok = mbar_wait(&bars[kBarXFree], (i - 1) & 1, abort_flag))) break;
+
+      if (warp == 1 && !AGG) {
+        // ---------------- query-side MMAs ----------------
+        auto issue_qk = [&](int i) -> bool {
+          const int st = i & 1;
+          if (!wait2(&bars[kBarKvFull + st], (i >> 1) & 1, &bars[kBarQFull], i & 1)) return false;
+          if (i > 0 && !mbar_wait(&bars[kBarXFree], (i - 1) & 1, abort_flag)) return false;
           tc_fence_after();
-          // S_qk = Q K^T  (both K-major, 64-byte swizzle)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_ss(tbase + kColX, smem_desc(stage + kOffQ + 32 * kk, 16, 512, kSw64),
-                   smem_desc(stage + kOffK + 32 * kk, 16, 512, kSw64), id_qk, kk);
+            mma_ss(tbase + kColX, adv(d_q, 32 * kk), adv(d_k_k, 8192 * st + 32 * kk), id_qk, kk);
           mma_commit(&bars[kBarSFull]);
+          return true;
+        };
+        if (nchunks > 0) ok = issue_qk(0);
+        for (int i = 0; ok && i < nchunks; ++i) {
+          const int st = i & 1;
           if (!(ok = mbar_wait(&bars[kBarPFull], i & 1, abort_flag))) break;
           tc_fence_after();
-          // O = P V  (P from TMEM)
+          // O = P V (P from tensor memory)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tbase + kColO, tbase + kColX + 8 * kk,
-                   smem_desc(stage + kOffV + 2048 * kk, 16384, 1024, kSw128), id_pv, kk);
-        }
-        if ((!AGG || i == 0) && !(ok = mbar_wait(&bars[kBarSnapFull], i & 1, abort_flag))) break;
-        tc_fence_after();
-        if (!AGG) {
+            mma_ts(tbase + kColO, tbase + kColX + 8 * kk, adv(d_v, 16384 * st + 2048 * kk), id_pv, kk);
           // U = Q Z_c
+          if (!(ok = mbar_wait(&bars[kBarZSnap], i & 1, abort_flag))) break;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_ss(tbase + kColU, smem_desc(stage + kOffQ + 32 * kk, 16, 512, kSw64),
-                   smem_desc(zsnap + 32 * kk, 16, 512, kSw64), id_u, kk);
-          // O += phi_q(Q) S_c, five feature slots
-          for (int s = 0; s < kTiles && ok; ++s, ++u) {
-            const int b = u & 1;
-            if (!(ok = mbar_wait(&bars[kBarSlotFull + b], (u >> 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            const uint32_t slot = slots + b * kSlotBytes;
-            const int nk = s == 4 ? 1 : 8;
-            for (int kk = 0; kk < nk; ++kk) {
-              const uint32_t a = slot + (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_ss(tbase + kColO, smem_desc(a, 16, 1024, kSw128),
-                     smem_desc(snap + (128 * s + 16 * kk) * 128, 16384, 1024, kSw128), id_ro, 1);
-            }
-            mma_commit(&bars[kBarSlotEmpty + b]);
+            mma_ss(tbase + kColU, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_u, kk);
+          mma_commit(&bars[kBarQEmpty]);
+          mma_commit(&bars[kBarZDone]);                  // Z_c snapshot no longer read
+          // O += phi_q(Q) S_c over nine 64-feature slots; slots 2m, 2m + 1
+          // read tile m of the snapshot once it is in place
+          for (int s9 = 0; s9 < kQSlots && ok; ++s9) {
+            const int u = i * kQSlots + s9, b = u & 1, m = s9 >> 1;
+            if ((s9 & 1) == 0)
+              ok = wait2(&bars[kBarTileSnap + m], i & 1, &bars[kBarQRingFull + b], (u >> 1) & 1);
+            else
+              ok = mbar_wait(&bars[kBarQRingFull + b], (u >> 1) & 1, abort_flag);
+            if (!ok) break;
+            const int nk = s9 == 8 ? 1 : 4;
+            for (int kk = 0; kk < nk; ++kk)
+              mma_ss(tbase + kColO, adv(d_qring, b * kQSlotBytes + 32 * kk),
+                     adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
+            mma_commit(&bars[kBarQRingEmpty + b]);
+            // tile m of the snapshot is no longer read after its last slot
+            if ((s9 & 1) == 1 || s9 == 8) mma_commit(&bars[kBarTileDone + m]);
           }
           if (!ok) break;
           mma_commit(&bars[kBarOFull]);
+          mma_commit(&bars[kBarKvEmpty + st]);          // this warp's reads of K_i, V_i are done
+          if (i + 1 < nchunks && !(ok = issue_qk(i + 1))) break;
         }
-        // S += phi(K)^T V, five feature tiles
-        for (int m = 0; m < kTiles && ok; ++m, ++u) {
-          const int b = u & 1;
-          if (!(ok = mbar_wait(&bars[kBarSlotFull + b], (u >> 1) & 1, abort_flag))) break;
+      } else if (warp == 10) {
+        // ---------------- state-side MMAs ----------------
+        for (int i = 0; ok && i < nchunks; ++i) {
+          const int st = i & 1;
+          if (!(ok = mbar_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
+          // the Z snapshot of this chunk's state has read Z in tensor memory
+          if ((!AGG || i == 0) && !(ok = mbar_wait(&bars[kBarZSnap], i & 1, abort_flag))) break;
           tc_fence_after();
-          const uint32_t slot = slots + b * kSlotBytes;
+          // Z += K^T K (A rows 32..127 alias other shared memory; unused lanes)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + kColS + 64 * m, smem_desc(slot + 2048 * kk, 16384, 1024, kSw128),
-                   smem_desc(stage + kOffV + 2048 * kk, 16384, 1024, kSw128), id_up, 1);
-          mma_commit(&bars[kBarSlotEmpty + b]);
-        }
-        if (!ok) break;
-        // Z += K^T K (A rows 32..127 alias other shared memory; unused lanes)
+            mma_ss(tbase + kColZ, adv(d_k_mn, 8192 * st + 1024 * kk),
+                   adv(d_k_mn, 8192 * st + 1024 * kk), id_z, 1);
+          if (!AGG) mma_commit(&bars[kBarZDone]);
+          // S tile m += phi(K)^T V, once the snapshot of tile m has read it
+          for (int m = 0; m < kTiles && ok; ++m) {
+            const int u = i * kTiles + m, b = u % NK;
+            uint64_t *full = &bars[kBarKRingFull + b];
+            const uint32_t par = (u / NK) & 1;
+            if (AGG) ok = mbar_wait(full, par, abort_flag);
+            else ok = wait2(&bars[kBarTileSnap + m], i & 1, full, par);
+            if (!ok) break;
+            if (!AGG) tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tbase + kColZ, smem_desc(stage + kOffK + 1024 * kk, 8192, 512, kSw64),
-                 smem_desc(stage + kOffK + 1024 * kk, 8192, 512, kSw64), id_z, 1);
-        mma_commit(&bars[kBarKvEmpty + st]);
-        if (!AGG || i == nchunks - 1) mma_commit(&bars[kBarUpdFull]);
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + kColS + 64 * m, adv(d_kring, b * kKSlotBytes + 2048 * kk),
+                     adv(d_v, 16384 * st + 2048 * kk), id_up, 1);
+            mma_commit(&bars[kBarKRingEmpty + b]);
+            if (!AGG) mma_commit(&bars[kBarTileDone + m]);
+          }
+          if (!ok) break;
+          mma_commit(&bars[kBarKvEmpty + st]);
+          if (i == nchunks - 1) mma_commit(&bars[kBarUpdFull]);
+        }
       }
     }
-  } else {
-    // ------------------------------------------------------------ math
+  } else if (warp < 6) {
+    // ------------------------------------------------ query side (warps 2..5)
+    if (!AGG) {
+      const int quarter = warp & 3;
+      const int r = quarter * 32 + lane;                  // TMEM lane = token of the chunk
+      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+      for (int i = 0; i < nchunks; ++i) {
+        const int c0 = t0 + i * kC;
+        if (!warp_wait(&bars[kBarQFull], i & 1, abort_flag)) break;
+        if (!warp_wait(&bars[kBarSFull], i & 1, abort_flag)) break;
+        tc_fence_after();
+        // ---- intra-chunk block: P = (Q K^T)^2 masked (key s <= min(r, T-1-c0)) ----
+        const int lim = min(r, T - 1 - c0);
+        float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t x[32];
+          tmem_ld32(tbase + lane_off + kColX + 32 * c, x);
+          tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int s0 = 32 * c + 2 * k;
+            const float2 a = make_float2(__uint_as_float(x[2 * k]), __uint_as_float(x[2 * k + 1]));
+            float2 w = __fmul2_rn(a, a);
+            w.x = s0 <= lim ? w.x : 0.f;
+            w.y = s0 + 1 <= lim ? w.y : 0.f;
+            lsum[k & 3] = __fadd2_rn(lsum[k & 3], w);
+            p[k] = pack_bf16x2(w.x, w.y);
+          }
+          tmem_st16(tbase + lane_off + kColX + 16 * c, p);
+        }
+        const float2 l01 = __fadd2_rn(lsum[0], lsum[1]), l23 = __fadd2_rn(lsum[2], lsum[3]);
+        const float2 lt = __fadd2_rn(l01, l23);
+        const float l_intra = lt.x + lt.y;
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(&bars[kBarPFull]);
+
+        // ---- phi_q(Q_c) into the ring, one slot per state tile ----
+        uint32_t XQ[16], P[32], P2[32];
+        load_pairs(smem + L::kOffQ, r, XQ, P);
+        warp_arrive(&bars[kBarQEmpty]);               // Q rows read
+#pragma unroll
+        for (int l = 0; l < 32; ++l) P2[l] = bmul2(P[l], 0x40004000u);   // x 2.0
+        bool ok = true;
+#pragma unroll
+        for (int s9 = 0; s9 < kQSlots; ++s9) {
+          const int u = i * kQSlots + s9;
+          if (ok) ok = ring_acquire(&bars[kBarQRingEmpty], 2, u);
+          if (ok) {
+            write_q_slot(qring + (u & 1) * kQSlotBytes, r, s9, P, P2);
+            ring_publish(&bars[kBarQRingFull], 2, u);
+          }
+        }
+        if (!ok) break;
+
+        // ---- epilogue: y = O / (l_intra + q^T U) ----
+        if (!warp_wait(&bars[kBarOFull], i & 1, abort_flag)) break;
+        tc_fence_after();
+        uint32_t uu[32], oo[32], oo2[32];
+        tmem_ld32(tbase + lane_off + kColU, uu);
+        tmem_ld32(tbase + lane_off + kColO, oo);
+        tmem_ld32(tbase + lane_off + kColO + 32, oo2);
+        tmem_wait_ld();
+        tc_fence_before();
+        warp_arrive(&bars[kBarXFree]);
+        float den = l_intra;
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+          const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162 *>(&XQ[w]);
+          den = fmaf(__low2float(qq), __uint_as_float(uu[2 * w]), den);
+          den = fmaf(__high2float(qq), __uint_as_float(uu[2 * w + 1]), den);
+        }
+        const int t = c0 + r;
+        if (!(den > 0.f) && t < T) flag_status(status, kStatusNonPositiveNormaliser);
+        if (t < T) {
+          const float inv = 1.f / den;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            oo[c] = __float_as_uint(__uint_as_float(oo[c]) * inv);
+            oo2[c] = __float_as_uint(__uint_as_float(oo2[c]) * inv);
+          }
+          uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * T + t) * kDV);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            dst[q4] = pack8(oo + 8 * q4);
+            dst[4 + q4] = pack8(oo2 + 8 * q4);
+          }
+        }
+      }
+    }
+  } else if (warp < 10) {
+    // -------------------------------------------------- key side (warps 6..9)
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;                    // TMEM lane / token / feature row
+    const int r = quarter * 32 + lane;                    // TMEM lane: token / feature row
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint8_t *snap = smem + kOffSnap;
-    uint8_t *zsnap = smem + kOffZSnap;
+    uint8_t *snap = smem + L::kOffSnap;
+    uint8_t *zsnap = smem + L::kOffZSnap;
     bool ok = true;
 
     // ---- carry-in: sum of the increments of segments 0 .. g-1 ----
@@ -342,17 +569,8 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
           for (int c = 0; c < 16; ++c) bits[c] = __float_as_uint(acc[c]);
           tmem_st16(tbase + lane_off + kColS + 64 * m + 16 * q4, bits);
           if (!AGG && f < kD) {
-            uint4 v0, v1;
-            v0.x = pack_bf16x2(acc[0], acc[1]);
-            v0.y = pack_bf16x2(acc[2], acc[3]);
-            v0.z = pack_bf16x2(acc[4], acc[5]);
-            v0.w = pack_bf16x2(acc[6], acc[7]);
-            v1.x = pack_bf16x2(acc[8], acc[9]);
-            v1.y = pack_bf16x2(acc[10], acc[11]);
-            v1.z = pack_bf16x2(acc[12], acc[13]);
-            v1.w = pack_bf16x2(acc[14], acc[15]);
-            *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4)) = v0;
-            *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4 + 1)) = v1;
+            *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4)) = pack8(bits);
+            *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4 + 1)) = pack8(bits + 8);
           }
         }
       }
@@ -374,157 +592,62 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         for (int c = 0; c < 16; ++c) bits[c] = __float_as_uint(acc[c]);
         tmem_st16(tbase + lane_off + kColZ + 16 * q2, bits);
         if (!AGG && r < kDK) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint4 v;
-            v.x = pack_bf16x2(acc[8 * h + 0], acc[8 * h + 1]);
-            v.y = pack_bf16x2(acc[8 * h + 2], acc[8 * h + 3]);
-            v.z = pack_bf16x2(acc[8 * h + 4], acc[8 * h + 5]);
-            v.w = pack_bf16x2(acc[8 * h + 6], acc[8 * h + 7]);
-            *reinterpret_cast<uint4 *>(zsnap + sw64(r, 2 * q2 + h)) = v;
-          }
+          *reinterpret_cast<uint4 *>(zsnap + sw64(r, 2 * q2)) = pack8(bits);
+          *reinterpret_cast<uint4 *>(zsnap + sw64(r, 2 * q2 + 1)) = pack8(bits + 8);
         }
       }
       fence_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[kBarSnapFull]);
+      warp_arrive(&bars[kBarZSnap]);
+      if (!AGG)
+        for (int m = 0; m < kTiles; ++m) warp_arrive(&bars[kBarTileSnap + m]);
     }
 
-    int u = 0;
     for (int i = 0; i < nchunks; ++i) {
       const int st = i & 1;
-      uint8_t *stage = smem + kOffStages + st * kStageBytes;
-      const int c0 = t0 + i * kC;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag));
-      if (!ok) break;
-      float l_intra = 0.f;
-      uint32_t XQ[16];
-      if (!AGG) {
-        // ---- intra-chunk block: P = (Q K^T)^2 masked, in place in TMEM ----
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarSFull], i & 1, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t x[32];
-          tmem_ld32(tbase + lane_off + kColX + 32 * c, x);
-          tmem_wait_ld();
-          uint32_t p[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int s0 = 32 * c + 2 * k;
-            const float a0 = __uint_as_float(x[2 * k]);
-            const float a1 = __uint_as_float(x[2 * k + 1]);
-            float w0 = a0 * a0, w1 = a1 * a1;
-            if (s0 > r || c0 + s0 >= T) w0 = 0.f;
-            if (s0 + 1 > r || c0 + s0 + 1 >= T) w1 = 0.f;
-            l_intra += w0 + w1;
-            p[k] = pack_bf16x2(w0, w1);
-          }
-          tmem_st16(tbase + lane_off + kColX + 16 * c, p);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars[kBarPFull]);
-
-        // ---- phi_q(Q_c) slots ----
-        uint32_t P[32], P2[32];
-        load_pairs(stage + kOffQ, r, XQ, P);
-#pragma unroll
-        for (int l = 0; l < 32; ++l) P2[l] = bmul2(P[l], 0x40004000u);   // x 2 (bf16 2.0)
-#pragma unroll
-        for (int s = 0; s < kTiles; ++s) {
-          const int us = u + s, b = us & 1;
-          if (ok && us >= 2)
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&bars[kBarSlotEmpty + b], ((us >> 1) - 1) & 1, abort_flag));
-          if (ok) {
-            write_phi_slot<true>(smem + kOffSlots + b * kSlotBytes, r, s, P, P2);
-            fence_async_smem();
-            mbar_arrive(&bars[kBarSlotFull + b]);
-          }
-        }
-        u += kTiles;
-        if (!ok) break;
-      }
-      // ---- phi(K_c) slots ----
+      if (!(ok = warp_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
+      // ---- phi(K_c) into the ring, one slot per state tile ----
       {
         uint32_t XK[16], P[32];
-        load_pairs(stage + kOffK, r, XK, P);
+        load_pairs(smem + L::kOffK + 8192 * st, r, XK, P);
+        warp_arrive(&bars[kBarKvEmpty + st]);         // K rows read
 #pragma unroll
-        for (int s = 0; s < kTiles; ++s) {
-          const int us = u + s, b = us & 1;
-          if (ok && us >= 2)
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&bars[kBarSlotEmpty + b], ((us >> 1) - 1) & 1, abort_flag));
-          if (ok) {
-            write_phi_slot<false>(smem + kOffSlots + b * kSlotBytes, r, s, P, P);
-            fence_async_smem();
-            mbar_arrive(&bars[kBarSlotFull + b]);
-          }
-        }
-        u += kTiles;
-        if (!ok) break;
-      }
-      mbar_arrive(&bars[kBarKvEmpty + st]);     // Q and K tiles no longer read here
-
-      if (!AGG) {
-        // ---- epilogue: y = (O) / (l_intra + q^T U) ----
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarOFull], i & 1, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t uu[32];
-        tmem_ld32(tbase + lane_off + kColU, uu);
-        uint32_t oo[32], oo2[32];
-        tmem_ld32(tbase + lane_off + kColO, oo);
-        tmem_ld32(tbase + lane_off + kColO + 32, oo2);
-        tmem_wait_ld();
-        float den = l_intra;
-#pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162 *>(&XQ[w]);
-          den = fmaf(__low2float(qq), __uint_as_float(uu[2 * w]), den);
-          den = fmaf(__high2float(qq), __uint_as_float(uu[2 * w + 1]), den);
-        }
-        tc_fence_before();
-        mbar_arrive(&bars[kBarXFree]);
-        const int t = c0 + r;
-        if (!(den > 0.f) && t < T) flag_status(status, kStatusNonPositiveNormaliser);
-        if (t < T) {
-          const float inv = 1.f / den;
-          uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * T + t) * kDV);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(oo[8 * q4 + 0]) * inv, __uint_as_float(oo[8 * q4 + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(oo[8 * q4 + 2]) * inv, __uint_as_float(oo[8 * q4 + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(oo[8 * q4 + 4]) * inv, __uint_as_float(oo[8 * q4 + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(oo[8 * q4 + 6]) * inv, __uint_as_float(oo[8 * q4 + 7]) * inv);
-            dst[q4] = v;
-          }
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(oo2[8 * q4 + 0]) * inv, __uint_as_float(oo2[8 * q4 + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(oo2[8 * q4 + 2]) * inv, __uint_as_float(oo2[8 * q4 + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(oo2[8 * q4 + 4]) * inv, __uint_as_float(oo2[8 * q4 + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(oo2[8 * q4 + 6]) * inv, __uint_as_float(oo2[8 * q4 + 7]) * inv);
-            dst[4 + q4] = v;
-          }
-        }
-      }
-
-      // ---- wait for S_c+1, Z_c+1 (increments only need the final state) ----
-      const bool last = i == nchunks - 1;
-      if (AGG && !last) continue;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars[kBarUpdFull], AGG ? 0 : (i & 1), abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      if (!last && !AGG) {
-        // snapshot S_c+1 -> bf16 B operand of the next readout; Z_c+1 likewise
         for (int m = 0; m < kTiles; ++m) {
-          if (m == 4 && quarter != 0) continue;          // tile 4: rows 512..527 (lanes 0..15)
+          const int u = i * kTiles + m;
+          if (ok) ok = ring_acquire(&bars[kBarKRingEmpty], NK, u);
+          if (ok) {
+            write_tile<false>(kring + (u % NK) * kKSlotBytes, r, m, P, P);
+            ring_publish(&bars[kBarKRingFull], NK, u);
+          }
+        }
+        if (!ok) break;
+      }
+      const bool last = i == nchunks - 1;
+      if (last) {
+        // the state after the last chunk is read below
+        if (!(ok = warp_wait(&bars[kBarUpdFull], 0, abort_flag))) break;
+        tc_fence_after();
+        continue;
+      }
+      if (AGG) continue;
+      // ---- snapshot Z_c+1, then S_c+1 tile by tile as the update finishes ----
+      if (!(ok = warp_wait(&bars[kBarZDone], i & 1, abort_flag))) break;
+      tc_fence_after();
+      if (quarter == 0) {
+        uint32_t zr[32];
+        tmem_ld32(tbase + lane_off + kColZ, zr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(zsnap + sw64(r, c)) = pack8(zr + 8 * c);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      warp_arrive(&bars[kBarZSnap]);
+      for (int m = 0; m < kTiles && ok; ++m) {
+        if (!(ok = warp_wait(&bars[kBarTileDone + m], i & 1, abort_flag))) break;
+        tc_fence_after();
+        if (m < 4 || quarter == 0) {                       // tile 4: rows 512..527 (lanes 0..15)
           const int f = 128 * m + r;
           uint32_t a[32], b2[32];
           tmem_ld32(tbase + lane_off + kColS + 64 * m, a);
@@ -533,39 +656,16 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
           if (f < kD) {
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(a[8 * q4 + 0]), __uint_as_float(a[8 * q4 + 1]));
-              v.y = pack_bf16x2(__uint_as_float(a[8 * q4 + 2]), __uint_as_float(a[8 * q4 + 3]));
-              v.z = pack_bf16x2(__uint_as_float(a[8 * q4 + 4]), __uint_as_float(a[8 * q4 + 5]));
-              v.w = pack_bf16x2(__uint_as_float(a[8 * q4 + 6]), __uint_as_float(a[8 * q4 + 7]));
-              *reinterpret_cast<uint4 *>(snap + sw128(f, q4)) = v;
-              uint4 v2;
-              v2.x = pack_bf16x2(__uint_as_float(b2[8 * q4 + 0]), __uint_as_float(b2[8 * q4 + 1]));
-              v2.y = pack_bf16x2(__uint_as_float(b2[8 * q4 + 2]), __uint_as_float(b2[8 * q4 + 3]));
-              v2.z = pack_bf16x2(__uint_as_float(b2[8 * q4 + 4]), __uint_as_float(b2[8 * q4 + 5]));
-              v2.w = pack_bf16x2(__uint_as_float(b2[8 * q4 + 6]), __uint_as_float(b2[8 * q4 + 7]));
-              *reinterpret_cast<uint4 *>(snap + sw128(f, 4 + q4)) = v2;
+              *reinterpret_cast<uint4 *>(snap + sw128(f, q4)) = pack8(a + 8 * q4);
+              *reinterpret_cast<uint4 *>(snap + sw128(f, 4 + q4)) = pack8(b2 + 8 * q4);
             }
-          }
-        }
-        if (quarter == 0) {
-          uint32_t zr[32];
-          tmem_ld32(tbase + lane_off + kColZ, zr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(zr[8 * c + 0]), __uint_as_float(zr[8 * c + 1]));
-            v.y = pack_bf16x2(__uint_as_float(zr[8 * c + 2]), __uint_as_float(zr[8 * c + 3]));
-            v.z = pack_bf16x2(__uint_as_float(zr[8 * c + 4]), __uint_as_float(zr[8 * c + 5]));
-            v.w = pack_bf16x2(__uint_as_float(zr[8 * c + 6]), __uint_as_float(zr[8 * c + 7]));
-            *reinterpret_cast<uint4 *>(zsnap + sw64(r, c)) = v;
           }
         }
         fence_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars[kBarSnapFull]);
+        warp_arrive(&bars[kBarTileSnap + m]);
       }
+      if (!ok) break;
     }
 
     // ---- state leaving the kernel ----
@@ -644,20 +744,22 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
   cudaError_t e;
   if (a.G > 1) {
     auto kagg = chunked_tc_kernel<true>;
-    e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Layout<true>::kSmemBytes);
     if (e != cudaSuccess) return e;
     ProfileScope prof("tc_segment_increment", a.stream);
-    kagg<<<(unsigned)(a.BH * (a.G - 1)), kThreads, kSmemBytes, a.stream>>>(
+    kagg<<<(unsigned)(a.BH * (a.G - 1)), kThreads, Layout<true>::kSmemBytes, a.stream>>>(
         tq, tk, tv, static_cast<__nv_bfloat16 *>(a.o), a.agg, nullptr, nullptr, a.status, a.T,
         a.G - 1, a.G, a.seg_len);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   auto kpass = chunked_tc_kernel<false>;
-  e = cudaFuncSetAttribute(kpass, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  e = cudaFuncSetAttribute(kpass, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Layout<false>::kSmemBytes);
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_segment_pass", a.stream);
-  kpass<<<(unsigned)(a.BH * a.G), kThreads, kSmemBytes, a.stream>>>(
+  kpass<<<(unsigned)(a.BH * a.G), kThreads, Layout<false>::kSmemBytes, a.stream>>>(
       tq, tk, tv, static_cast<__nv_bfloat16 *>(a.o), a.agg, a.S_out, a.z_out, a.status, a.T, a.G,
       a.G, a.seg_len);
   return cudaGetLastError();

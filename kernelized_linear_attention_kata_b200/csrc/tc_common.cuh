@@ -12,9 +12,18 @@
 namespace kata {
 namespace tc {
 
-// A bounded wait gives up after this many polls, raises the CTA's abort flag
-// and reports failure; nothing in these kernels spins forever.
-constexpr uint32_t kSpinLimit = 1u << 26;
+// A bounded wait gives up after kWaitLimitNs of wall-clock time (read from
+// %globaltimer), raises the CTA's abort flag and reports failure; nothing in
+// these kernels waits forever.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;       // 2 s
+// Longest time one try_wait may suspend the thread before it re-checks.
+constexpr uint32_t kSuspendHintNs = 1000000u;          // 1 ms
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -41,11 +50,26 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+// One test of the phase; the thread may sleep up to `hint_ns` waiting for it
+// and is woken as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of the phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -54,15 +78,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Gives up (returns
-// false and raises *abort) after kSpinLimit polls, or returns false at once
-// if another thread of the CTA has already raised *abort.
+// false and raises *abort) after kWaitLimitNs, or returns false at once if
+// another thread of the CTA has already raised *abort.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 1023u && *abort) return false;
+  if (mbar_test_wait(bar, parity)) return true;           // already complete: no suspend
+  if (mbar_try_wait(bar, parity, kSuspendHintNs)) return true;
+  const uint64_t start = global_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity, kSuspendHintNs)) return true;
+    if (*abort) return false;
+    if (global_ns() - start > kWaitLimitNs) {
+      *abort = 1;
+      return false;
+    }
   }
-  *abort = 1;
-  return false;
 }
 
 // Orders this thread's generic-proxy shared-memory writes before later
