@@ -25,24 +25,30 @@
 // leaves the kernel (S_out, z_out).
 //
 // Warp roles (352 threads): warp 0 TMA producer; warp 1 TMEM allocation and
-// the query-side MMAs (Q K^T, P V, U, the readout into O); warp 10 the
+// the query-side MMAs (Q K^T, P V, the readout into O); warp 10 the
 // state-side MMAs (the update of S and Z) - two issuing threads so that one's
 // waits are covered by the other's MMAs; warps 2-5, the query side: the
-// intra-chunk P, the query features into the ring, the epilogue; warps 6-9,
-// the key side: the key features into the ring, the bf16 snapshot of the
-// state after each update, the carry-in and the state written out. Math
-// thread r owns TMEM lane r (quarter = warp mod 4): token r of the chunk for
-// the token-major tiles, feature row r of each 128-feature state tile.
+// intra-chunk P, the query features into tensor memory, the epilogue (y
+// staged in shared memory, written by one TMA store per chunk); warps 6-9,
+// the key side: the key features into the shared-memory ring, the bf16
+// snapshot of the state after each update, the carry-in and the state
+// written out. Math thread r owns TMEM lane r (quarter = warp mod 4):
+// token r of the chunk for the token-major tiles, feature row r of each
+// 128-feature state tile.
 //
 // Tensor memory (512 columns, fp32):
 //   [  0, 320)  S, five 128-feature tiles of 64 columns (tile 4: 16 rows used)
 //   [320, 352)  Z (lanes 0..31)
-//   [352, 384)  U = Q_c Z_c (den of the inter-chunk part)
-//   [384, 512)  Q_c K_c^T; then P (bf16, in place, [384, 448)) and O ([448, 512))
-// Shared memory (220 KB): the Q tile (single buffer), two TMA stages of K and
-// V, the bf16 snapshot of S_c (the readout's B operand) and of Z_c, and a
-// ring of three 128-feature slots shared by the query features (readout A
-// operand) and the key features (update A operand).
+//   [352, 384)  U = Q_c Z_c (den of the inter-chunk part: q^T Z_c q = q . u);
+//               once read, query-feature slot 0 (64 bf16 features per token)
+//   [384, 512)  Q_c K_c^T; then P (bf16, in place, [384, 448)) and O ([448, 512));
+//               once P V is done, [384, 416) and [416, 448) are query slots 1, 2
+// The readout takes its A operand (the query features) from tensor memory,
+// so the only shared-memory operands of the hot loop are the key features
+// and the state snapshot.
+// Shared memory (206 KB): the Q tile (single buffer), two TMA stages of K and
+// V, the bf16 snapshots of S_c (the readout's B operand) and Z_c, the output
+// stage and a ring of two 128-feature key slots (the update's A operand).
 #include "common.cuh"
 #include "launch.h"
 #include "profile.h"
@@ -61,21 +67,24 @@ constexpr int kD = 528;
 constexpr int kTiles = 5;          // 128-feature state tiles: ceil(528 / 128)
 constexpr int kThreads = 352;      // 11 warps
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColZ = 320, kColU = 352, kColX = 384, kColO = 448;
+constexpr uint32_t kColS = 0, kColZ = 320, kColX = 384, kColO = 448;
+constexpr uint32_t kColRing = 352;  // query slot b at kColRing + 32 b (b = 0, 1, 2); U in slot 0
+constexpr int kRing = 3;
+// Ring entry of readout slot s9: entries 1, 2 (P's columns) take the first
+// two slots of a chunk, entry 0 (U's columns) the third, and so on.
+__host__ __device__ constexpr int ring_entry(int s9) { return (s9 + 1) % kRing; }
 constexpr int kAggFloats = kD * kDV + kDK * kDK;      // one segment increment
 
-// Shared memory layout (bytes from a 1024-aligned base). Features travel
-// through two rings, each with one producer set and one consumer warp (an
-// mbarrier parity wait is only unambiguous for a single consumer in order):
-//   query ring: 16 KB slots of 128 token rows x 64 query features (readout
-//               A operand, K-major), nine uses per chunk;
-//   key ring:   32 KB slots of 128 token rows x 128 key features, as two
-//               64-feature groups 16 KB apart (update A operand, MN-major),
-//               five uses per chunk, one per state tile.
+// Shared memory layout (bytes from a 1024-aligned base). Key features travel
+// through a ring with one producer set and one consumer warp (an mbarrier
+// parity wait is only unambiguous for a single consumer in order): 32 KB
+// slots of 128 token rows x 128 key features, as two 64-feature groups 16 KB
+// apart (update A operand, MN-major), five uses per chunk, one per state tile.
 //   forward pass:  Q 8 KB | K 2 x 8 KB | V 2 x 16 KB | S_c bf16 66 KB |
-//                  Z_c bf16 2 KB | query ring 2 x 16 KB | key ring 2 x 32 KB
+//                  Z_c bf16 2 KB | y stage 16 KB | key ring 2 x 32 KB
 //   increments:    K 2 x 8 KB | V 2 x 16 KB | key ring 5 x 32 KB
-constexpr int kQSlotBytes = 16384;
+// The query features travel through a ring of three tensor-memory slots
+// (readout A operand), nine uses per chunk (64 features each).
 constexpr int kKSlotBytes = 32768;
 constexpr int kQSlots = 9;          // 64-feature readout slots per chunk
 template <bool AGG>
@@ -84,23 +93,23 @@ struct Layout {
   static constexpr int kOffK = AGG ? 0 : 8192;
   static constexpr int kOffV = kOffK + 16384;
   static constexpr int kOffSnap = kOffV + 32768;      // [528][64] bf16, 128 B rows (pass only)
-  static constexpr int kOffZSnap = kOffSnap + (AGG ? 0 : kD * 128);
-  static constexpr int kOffQRing = kOffZSnap + (AGG ? 0 : 2048);
-  static constexpr int kQRingSlots = AGG ? 0 : 2;
-  static constexpr int kOffKRing = kOffQRing + kQRingSlots * kQSlotBytes;
+  static constexpr int kOffZSnap = kOffSnap + (AGG ? 0 : kD * 128);   // [32][32] bf16, 64 B rows
+  static constexpr int kOffStage = kOffZSnap + (AGG ? 0 : 2048);      // y: [128][64] bf16, 128 B rows
+  static constexpr int kOffKRing = kOffStage + (AGG ? 0 : 16384);
   static constexpr int kKRingSlots = AGG ? 5 : 2;
   static constexpr int kOffBars = kOffKRing + kKRingSlots * kKSlotBytes;
   static constexpr int kSmemBytes = kOffBars + 1024 + 1024;   // barriers + alignment slack
   static_assert(kOffV % 1024 == 0 && kOffSnap % 1024 == 0 && kOffZSnap % 1024 == 0 &&
-                kOffQRing % 1024 == 0 && kOffKRing % 1024 == 0,
+                    kOffStage % 1024 == 0 && kOffKRing % 1024 == 0,
                 "swizzle atoms need 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 enum {
   kBarQFull = 0, kBarQEmpty, kBarKvFull, kBarKvEmpty = kBarKvFull + 2, kBarSFull = kBarKvEmpty + 2,
-  kBarPFull, kBarOFull, kBarXFree, kBarUpdFull, kBarZDone, kBarZSnap, kBarTileDone,
-  kBarTileSnap = kBarTileDone + 5, kBarQRingFull = kBarTileSnap + 5, kBarQRingEmpty = kBarQRingFull + 2,
-  kBarKRingFull = kBarQRingEmpty + 2, kBarKRingEmpty = kBarKRingFull + 5, kNumBars = kBarKRingEmpty + 5
+  kBarPFull, kBarPVDone, kBarUDone, kBarOFull, kBarXFree, kBarUpdFull, kBarZDone, kBarZSnap,
+  kBarStageFull, kBarStageFree, kBarTileDone,
+  kBarTileSnap = kBarTileDone + 5, kBarRingFull = kBarTileSnap + 5, kBarRingEmpty = kBarRingFull + kRing,
+  kBarKRingFull = kBarRingEmpty + kRing, kBarKRingEmpty = kBarKRingFull + 5, kNumBars = kBarKRingEmpty + 5
 };
 constexpr int kBarBytes = 8 * kNumBars;
 static_assert(kBarBytes + 8 <= 1024, "barrier area");
@@ -136,49 +145,60 @@ __device__ __forceinline__ int abi_row(int f) {
   return i * kDK - i * (i - 1) / 2 + (j - i);
 }
 
-// One 16-byte chunk (8 features (d, l0 .. l0+7)) of a token's feature row.
-// P[l] holds the bf16 pair (x_l, x_(l+1) mod 32); M is P, or P doubled for
-// the query's off-diagonal multiplicity.
-__device__ __forceinline__ uint4 phi_chunk(int d, int l0, const uint32_t (&P)[32],
-                                           const uint32_t (&M)[32]) {
-  uint32_t w[4];
+// The feature loops below are rolled (one body for every slot or tile, to
+// keep the code small); register indices stay static by walking a rotated
+// copy R of the pair array: R[l] = P[(l + d0) mod 32] for the slot's or
+// tile's first offset d0, rotated further after each use.
+__device__ __forceinline__ void rotate_left(uint32_t (&R)[32], int by) {
+  uint32_t t[32];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int l = l0 + 2 * k;
-    w[k] = bmul2(P[l], M[(l + d) & 31]);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+  for (int l = 0; l < 32; ++l) t[l] = R[(l + by) & 31];
+#pragma unroll
+  for (int l = 0; l < 32; ++l) R[l] = t[l];
 }
 
-// Query features of readout slot s (features 64 s .. 64 s + 63, offsets
-// d = 2 s, 2 s + 1; slot 8 holds only (16, l < 16)) for one token row, with
-// the off-diagonal multiplicity 2 (P2 = 2 P).
-__device__ __forceinline__ void write_q_slot(uint8_t *slot, int row, int s, const uint32_t (&P)[32],
-                                             const uint32_t (&P2)[32]) {
+// Query features of readout slot s (features 64 s .. 64 s + 63: offsets
+// d = 2 s, 2 s + 1; slot 8 holds only (16, l < 16)) for one token row, as 32
+// bf16 pairs, word c holding features 2c (low half) and 2c + 1 (the K order
+// of a tensor-memory A operand): word j = (2 s, 2 j), word 16 + j =
+// (2 s + 1, 2 j). R = P rotated by 2 s. The off-diagonal multiplicity 2 of
+// the query feature is carried by the state instead (see write_tile).
+__device__ __forceinline__ void q_slot_words(const uint32_t (&P)[32], const uint32_t (&R)[32],
+                                             bool partial, uint32_t (&w)[32]) {
 #pragma unroll
-  for (int cc = 0; cc < 8; ++cc) {
-    if (s == 8 && cc >= 2) continue;
-    const int d = 2 * s + (cc >> 2);
-    const uint4 v = d == 0 ? phi_chunk(d, (cc & 3) * 8, P, P) : phi_chunk(d, (cc & 3) * 8, P, P2);
-    *reinterpret_cast<uint4 *>(slot + sw128(row, cc)) = v;
+  for (int j = 0; j < 16; ++j) {
+    w[j] = bmul2(P[2 * j], R[2 * j]);
+    w[16 + j] = bmul2(P[2 * j], R[2 * j + 1]);
+  }
+  if (partial) {
+#pragma unroll
+    for (int j = 8; j < 32; ++j) w[j] = 0u;
   }
 }
 
-// Features of state tile m (128 m .. 128 m + 127; two 64-feature groups 16
-// KB apart; tile 4 holds only (16, l < 16)) for one token row. QUERY doubles
-// the off-diagonal features (the readout side).
-template <bool QUERY>
-__device__ __forceinline__ void write_tile(uint8_t *slot, int row, int m, const uint32_t (&P)[32],
-                                           const uint32_t (&P2)[32]) {
+// Key features of state tile m (128 m .. 128 m + 127: offsets d = 4 m ..
+// 4 m + 3 in two 64-feature groups 16 KB apart; tile 4 holds only
+// (16, l < 16)) for one token row, with the off-diagonal features doubled:
+// R2 = 2 P rotated by 4 m, and the diagonal (tile 0, first offset) scaled
+// back by dscale = 1/2. The state accumulated inside the kernel is therefore
+// S'_f = m_f S_f (m_f = 1 on the diagonal, 2 off it), so that the readout's
+// plain query products give phi_q(q) . S; the scaling by 2 is exact and is
+// undone where the state leaves the kernel.
+__device__ __forceinline__ void write_tile(uint8_t *slot, int row, bool partial, uint32_t dscale,
+                                           const uint32_t (&P)[32], const uint32_t (&R2)[32]) {
 #pragma unroll
   for (int g2 = 0; g2 < 2; ++g2) {
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
-      if (m == 4 && (g2 != 0 || cc >= 2)) continue;
-      const int d = 4 * m + 2 * g2 + (cc >> 2);
-      const uint4 v = (QUERY && d != 0) ? phi_chunk(d, (cc & 3) * 8, P, P2)
-                                        : phi_chunk(d, (cc & 3) * 8, P, P);
-      *reinterpret_cast<uint4 *>(slot + g2 * 16384 + sw128(row, cc)) = v;
+      if (partial && (g2 != 0 || cc >= 2)) continue;
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int l = 8 * (cc & 3) + 2 * k;
+        w[k] = bmul2(P[l], R2[(l + 2 * g2 + (cc >> 2)) & 31]);
+        if (g2 == 0 && cc < 4) w[k] = bmul2(w[k], dscale);
+      }
+      *reinterpret_cast<uint4 *>(slot + g2 * 16384 + sw128(row, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }
@@ -219,7 +239,7 @@ __device__ __forceinline__ void warp_arrive(uint64_t *bar) { mbar_arrive(bar); }
 template <bool AGG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmv, __nv_bfloat16 *__restrict__ o,
+                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                   float *__restrict__ agg, float *__restrict__ S_out, float *__restrict__ z_out,
                   unsigned *__restrict__ status, int T, int G_grid, int G_total, int seg_len) {
   using L = Layout<AGG>;
@@ -244,13 +264,17 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     // kSetArrivals for the threads of a math set
     constexpr uint32_t A = kSetArrivals;
     mbar_init(&bars[kBarQFull], 1);
-    mbar_init(&bars[kBarQEmpty], 1 + A);
+    mbar_init(&bars[kBarQEmpty], 1 + A);            // Q K^T commit + query side
     for (int st = 0; st < 2; ++st) {
       mbar_init(&bars[kBarKvFull + st], 1);
       mbar_init(&bars[kBarKvEmpty + st], (AGG ? 1 : 2) + A);   // MMA warp(s) + key side
     }
     mbar_init(&bars[kBarSFull], 1);
     mbar_init(&bars[kBarPFull], A);
+    mbar_init(&bars[kBarPVDone], 1);
+    mbar_init(&bars[kBarUDone], 1);
+    mbar_init(&bars[kBarStageFull], A);
+    mbar_init(&bars[kBarStageFree], 1);
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarXFree], A);
     mbar_init(&bars[kBarUpdFull], 1);
@@ -262,9 +286,9 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       mbar_init(&bars[kBarTileDone + m], 2);
       mbar_init(&bars[kBarTileSnap + m], A);
     }
-    for (int k = 0; k < 2; ++k) {
-      mbar_init(&bars[kBarQRingFull + k], A);
-      mbar_init(&bars[kBarQRingEmpty + k], 1);
+    for (int k = 0; k < kRing; ++k) {
+      mbar_init(&bars[kBarRingFull + k], A);
+      mbar_init(&bars[kBarRingEmpty + k], 1);
     }
     for (int k = 0; k < NK; ++k) {
       mbar_init(&bars[kBarKRingFull + k], A);
@@ -281,7 +305,6 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  uint8_t *qring = smem + L::kOffQRing;
   uint8_t *kring = smem + L::kOffKRing;
 
   // Producer side of a ring (one math warp set): use u of a ring with n
@@ -299,7 +322,10 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     if (lane == 0) {
       tma_prefetch_desc(&tmk);
       tma_prefetch_desc(&tmv);
-      if (!AGG) tma_prefetch_desc(&tmq);
+      if (!AGG) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmo);
+      }
       for (int i = 0; i < nchunks; ++i) {
         const int st = i & 1;
         const int row = t0 + i * kC;
@@ -318,7 +344,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     // ------------------------------------------------------------ MMA issue
     // Two issuing warps with independent accumulators, so that one's waits
     // are covered by the other's MMAs: warp 1 issues the query side (Q K^T,
-    // P V, U, the readout into O); warp 10 issues the state side (the update
+    // P V, the readout into O); warp 10 issues the state side (the update
     // of S and Z).
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 128, false, false);
@@ -328,21 +354,20 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       constexpr uint32_t id_up = idesc_bf16(128, kDV, true, true);
       constexpr uint32_t id_z = idesc_bf16(128, 32, true, true);
       const uint32_t qa = smem_u32(smem + L::kOffQ);
-      const uint32_t qring_a = smem_u32(qring), kring_a = smem_u32(kring);
+      const uint32_t kring_a = smem_u32(kring);
       // Descriptors are built once; operands at other offsets of the same
       // layout differ only in the start-address field (bytes / 16).
       auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
       const uint64_t d_q = smem_desc(qa, 16, 512, kSw64);                       // Q, K-major
       const uint64_t d_z = smem_desc(smem_u32(smem + L::kOffZSnap), 16, 512, kSw64);
       const uint64_t d_snap = smem_desc(smem_u32(smem + L::kOffSnap), 16384, 1024, kSw128);
-      const uint64_t d_qring = smem_desc(qring_a, 16, 1024, kSw128);            // readout A
       const uint64_t d_kring = smem_desc(kring_a, 16384, 1024, kSw128);         // update A
       const uint64_t d_k_k = smem_desc(smem_u32(smem + L::kOffK), 16, 512, kSw64);     // K, K-major
       const uint64_t d_k_mn = smem_desc(smem_u32(smem + L::kOffK), 8192, 512, kSw64);  // K, MN-major
       const uint64_t d_v = smem_desc(smem_u32(smem + L::kOffV), 16384, 1024, kSw128);  // V, MN-major
-      // Ring slots are shared memory written by threads (ordered for the
-      // tensor core by their proxy fence and the mbarrier), so ring waits
-      // need no tcgen05 fence; only hand-offs of tensor memory do.
+      // Key-ring slots are shared memory written by threads (ordered for the
+      // tensor core by their proxy fence and the mbarrier), so their waits
+      // need no tcgen05 fence; hand-offs of tensor memory do.
       // Two barriers tested back to back so that their latencies overlap.
       auto wait2 = [&](uint64_t *b1, uint32_t p1, uint64_t *b2, uint32_t p2) -> bool {
         const bool a = mbar_test_wait(b1, p1), b = mbar_test_wait(b2, p2);
@@ -353,10 +378,19 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 
       if (warp == 1 && !AGG) {
         // ---------------- query-side MMAs ----------------
+        // Every test of a barrier by an issuing thread drains its MMAs from
+        // the tensor pipe, so the issuing threads wait on as few barriers as
+        // possible: the math warps wait on the others first and fold them
+        // into their own arrivals (XFree implies Q_i+1 and K_i+1, V_i+1 in
+        // shared memory; PFull implies the Z_c snapshot; a ring slot implies
+        // the snapshot tile it is read against).
         auto issue_qk = [&](int i) -> bool {
           const int st = i & 1;
-          if (!wait2(&bars[kBarKvFull + st], (i >> 1) & 1, &bars[kBarQFull], i & 1)) return false;
-          if (i > 0 && !mbar_wait(&bars[kBarXFree], (i - 1) & 1, abort_flag)) return false;
+          if (i == 0) {
+            if (!wait2(&bars[kBarKvFull + st], (i >> 1) & 1, &bars[kBarQFull], i & 1)) return false;
+          } else if (!mbar_wait(&bars[kBarXFree], (i - 1) & 1, abort_flag)) {
+            return false;
+          }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
@@ -373,27 +407,26 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tbase + kColO, tbase + kColX + 8 * kk, adv(d_v, 16384 * st + 2048 * kk), id_pv, kk);
-          // U = Q Z_c
-          if (!(ok = mbar_wait(&bars[kBarZSnap], i & 1, abort_flag))) break;
+          mma_commit(&bars[kBarPVDone]);                 // P's columns become query slots 1, 2
+          // U = Q Z_c into query slot 0
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_ss(tbase + kColU, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_u, kk);
-          mma_commit(&bars[kBarQEmpty]);
+            mma_ss(tbase + kColRing, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_u, kk);
+          mma_commit(&bars[kBarUDone]);
+          mma_commit(&bars[kBarQEmpty]);                 // Q tile no longer read by the tensor core
           mma_commit(&bars[kBarZDone]);                  // Z_c snapshot no longer read
-          // O += phi_q(Q) S_c over nine 64-feature slots; slots 2m, 2m + 1
-          // read tile m of the snapshot once it is in place
+          // O += phi_q(Q) S_c over nine 64-feature slots (slot s9 in ring
+          // entry ring_entry(s9), A from tensor memory); slots 2m, 2m + 1 read
+          // tile m of the snapshot once it is in place
           for (int s9 = 0; s9 < kQSlots && ok; ++s9) {
-            const int u = i * kQSlots + s9, b = u & 1, m = s9 >> 1;
-            if ((s9 & 1) == 0)
-              ok = wait2(&bars[kBarTileSnap + m], i & 1, &bars[kBarQRingFull + b], (u >> 1) & 1);
-            else
-              ok = mbar_wait(&bars[kBarQRingFull + b], (u >> 1) & 1, abort_flag);
-            if (!ok) break;
+            const int b = ring_entry(s9), k = kRing * i + s9 / kRing, m = s9 >> 1;
+            if (!(ok = mbar_wait(&bars[kBarRingFull + b], k & 1, abort_flag))) break;
+            tc_fence_after();
             const int nk = s9 == 8 ? 1 : 4;
+            const uint32_t a_col = tbase + kColRing + 32 * b;
             for (int kk = 0; kk < nk; ++kk)
-              mma_ss(tbase + kColO, adv(d_qring, b * kQSlotBytes + 32 * kk),
-                     adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
-            mma_commit(&bars[kBarQRingEmpty + b]);
+              mma_ts(tbase + kColO, a_col + 8 * kk, adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
+            mma_commit(&bars[kBarRingEmpty + b]);
             // tile m of the snapshot is no longer read after its last slot
             if ((s9 & 1) == 1 || s9 == 8) mma_commit(&bars[kBarTileDone + m]);
           }
@@ -404,27 +437,24 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         }
       } else if (warp == 10) {
         // ---------------- state-side MMAs ----------------
+        // The key side writes the key features of chunk i after its snapshots
+        // of S_i and Z_i (and after K_i, V_i arrived), so a full key-ring slot
+        // also says that the state it updates has been read.
         for (int i = 0; ok && i < nchunks; ++i) {
           const int st = i & 1;
-          if (!(ok = mbar_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
-          // the Z snapshot of this chunk's state has read Z in tensor memory
-          if ((!AGG || i == 0) && !(ok = mbar_wait(&bars[kBarZSnap], i & 1, abort_flag))) break;
-          tc_fence_after();
-          // Z += K^T K (A rows 32..127 alias other shared memory; unused lanes)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + kColZ, adv(d_k_mn, 8192 * st + 1024 * kk),
-                   adv(d_k_mn, 8192 * st + 1024 * kk), id_z, 1);
-          if (!AGG) mma_commit(&bars[kBarZDone]);
-          // S tile m += phi(K)^T V, once the snapshot of tile m has read it
           for (int m = 0; m < kTiles && ok; ++m) {
             const int u = i * kTiles + m, b = u % NK;
-            uint64_t *full = &bars[kBarKRingFull + b];
-            const uint32_t par = (u / NK) & 1;
-            if (AGG) ok = mbar_wait(full, par, abort_flag);
-            else ok = wait2(&bars[kBarTileSnap + m], i & 1, full, par);
-            if (!ok) break;
-            if (!AGG) tc_fence_after();
+            if (!(ok = mbar_wait(&bars[kBarKRingFull + b], (u / NK) & 1, abort_flag))) break;
+            tc_fence_after();
+            if (m == 0) {
+              // Z += K^T K (A rows 32..127 alias other shared memory; unused lanes)
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tbase + kColZ, adv(d_k_mn, 8192 * st + 1024 * kk),
+                       adv(d_k_mn, 8192 * st + 1024 * kk), id_z, 1);
+              if (!AGG) mma_commit(&bars[kBarZDone]);
+            }
+            // S tile m += phi(K)^T V
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tbase + kColS + 64 * m, adv(d_kring, b * kKSlotBytes + 2048 * kk),
@@ -444,92 +474,147 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       const int quarter = warp & 3;
       const int r = quarter * 32 + lane;                  // TMEM lane = token of the chunk
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+      uint8_t *stage = smem + L::kOffStage;
       for (int i = 0; i < nchunks; ++i) {
         const int c0 = t0 + i * kC;
         if (!warp_wait(&bars[kBarQFull], i & 1, abort_flag)) break;
         if (!warp_wait(&bars[kBarSFull], i & 1, abort_flag)) break;
         tc_fence_after();
         // ---- intra-chunk block: P = (Q K^T)^2 masked (key s <= min(r, T-1-c0)) ----
+        // 64 columns per tensor-memory wait; P (bf16) overwrites the columns
+        // already read
         const int lim = min(r, T - 1 - c0);
         float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t x[32];
-          tmem_ld32(tbase + lane_off + kColX + 32 * c, x);
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t x[2][32];
+          tmem_ld32(tbase + lane_off + kColX + 64 * h, x[0]);
+          tmem_ld32(tbase + lane_off + kColX + 64 * h + 32, x[1]);
           tmem_wait_ld();
-          uint32_t p[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int s0 = 32 * c + 2 * k;
-            const float2 a = make_float2(__uint_as_float(x[2 * k]), __uint_as_float(x[2 * k + 1]));
-            float2 w = __fmul2_rn(a, a);
-            w.x = s0 <= lim ? w.x : 0.f;
-            w.y = s0 + 1 <= lim ? w.y : 0.f;
-            lsum[k & 3] = __fadd2_rn(lsum[k & 3], w);
-            p[k] = pack_bf16x2(w.x, w.y);
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int c = 2 * h + c2;
+            uint32_t p[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const int s0 = 32 * c + 2 * k;
+              const float2 a =
+                  make_float2(__uint_as_float(x[c2][2 * k]), __uint_as_float(x[c2][2 * k + 1]));
+              float2 w = __fmul2_rn(a, a);
+              w.x = s0 <= lim ? w.x : 0.f;
+              w.y = s0 + 1 <= lim ? w.y : 0.f;
+              lsum[k & 3] = __fadd2_rn(lsum[k & 3], w);
+              p[k] = pack_bf16x2(w.x, w.y);
+            }
+            tmem_st16(tbase + lane_off + kColX + 16 * c, p);
           }
-          tmem_st16(tbase + lane_off + kColX + 16 * c, p);
         }
         const float2 l01 = __fadd2_rn(lsum[0], lsum[1]), l23 = __fadd2_rn(lsum[2], lsum[3]);
         const float2 lt = __fadd2_rn(l01, l23);
         const float l_intra = lt.x + lt.y;
         tmem_wait_st();
         tc_fence_before();
+        // PFull also hands over the Z_c snapshot (read by U after P V)
+        if (!warp_wait(&bars[kBarZSnap], i & 1, abort_flag)) break;
         warp_arrive(&bars[kBarPFull]);
 
-        // ---- phi_q(Q_c) into the ring, one slot per state tile ----
-        uint32_t XQ[16], P[32], P2[32];
+        // ---- phi_q(Q_c) into the tensor-memory ring, 64 features a slot ----
+        uint32_t XQ[16], P[32];
         load_pairs(smem + L::kOffQ, r, XQ, P);
         warp_arrive(&bars[kBarQEmpty]);               // Q rows read
-#pragma unroll
-        for (int l = 0; l < 32; ++l) P2[l] = bmul2(P[l], 0x40004000u);   // x 2.0
         bool ok = true;
+        float den_inter = 0.f;
+        uint32_t R[32];
 #pragma unroll
+        for (int l = 0; l < 32; ++l) R[l] = P[l];
+#pragma unroll 1
         for (int s9 = 0; s9 < kQSlots; ++s9) {
-          const int u = i * kQSlots + s9;
-          if (ok) ok = ring_acquire(&bars[kBarQRingEmpty], 2, u);
+          const int b = ring_entry(s9), j = s9 / kRing, k = kRing * i + j;
+          // Entry b may be written once its previous use has been read. The
+          // first use of a chunk instead waits for what last used the columns
+          // in this chunk (P V for entries 1 and 2, U for entry 0), which
+          // also implies every use of the previous chunk is complete; entry 0
+          // first hands its U to the denominator.
           if (ok) {
-            write_q_slot(qring + (u & 1) * kQSlotBytes, r, s9, P, P2);
-            ring_publish(&bars[kBarQRingFull], 2, u);
+            if (j == 0 && b == 1) {
+              ok = warp_wait(&bars[kBarPVDone], i & 1, abort_flag);
+            } else if (j == 0 && b == 0) {
+              ok = warp_wait(&bars[kBarUDone], i & 1, abort_flag);
+              if (ok) {
+                tc_fence_after();
+                uint32_t uu[32];
+                tmem_ld32(tbase + lane_off + kColRing, uu);
+                tmem_wait_ld();
+#pragma unroll
+                for (int w = 0; w < 16; ++w) {
+                  const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162 *>(&XQ[w]);
+                  den_inter = fmaf(__low2float(qq), __uint_as_float(uu[2 * w]), den_inter);
+                  den_inter = fmaf(__high2float(qq), __uint_as_float(uu[2 * w + 1]), den_inter);
+                }
+              }
+            } else if (j > 0) {
+              ok = warp_wait(&bars[kBarRingEmpty + b], (k - 1) & 1, abort_flag);
+            }
           }
+          // the slot is read against snapshot tile s9 / 2 of S_c
+          if (ok && (s9 & 1) == 0) ok = warp_wait(&bars[kBarTileSnap + (s9 >> 1)], i & 1, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            uint32_t w[32];
+            q_slot_words(P, R, s9 == kQSlots - 1, w);
+            tmem_st32(tbase + lane_off + kColRing + 32 * b, w);
+            tmem_wait_st();
+            tc_fence_before();
+            warp_arrive(&bars[kBarRingFull + b]);
+          }
+          rotate_left(R, 2);
         }
         if (!ok) break;
 
-        // ---- epilogue: y = O / (l_intra + q^T U) ----
+        // ---- epilogue: y = O / (l_intra + q^T Z_c q) ----
         if (!warp_wait(&bars[kBarOFull], i & 1, abort_flag)) break;
         tc_fence_after();
-        uint32_t uu[32], oo[32], oo2[32];
-        tmem_ld32(tbase + lane_off + kColU, uu);
+        uint32_t oo[32], oo2[32];
         tmem_ld32(tbase + lane_off + kColO, oo);
         tmem_ld32(tbase + lane_off + kColO + 32, oo2);
         tmem_wait_ld();
         tc_fence_before();
+        // XFree also hands over Q_c+1 and K_c+1, V_c+1 (read by its Q K^T)
+        if (i + 1 < nchunks &&
+            !(warp_wait(&bars[kBarQFull], (i + 1) & 1, abort_flag) &&
+              warp_wait(&bars[kBarKvFull + ((i + 1) & 1)], ((i + 1) >> 1) & 1, abort_flag)))
+          break;
         warp_arrive(&bars[kBarXFree]);
-        float den = l_intra;
-#pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162 *>(&XQ[w]);
-          den = fmaf(__low2float(qq), __uint_as_float(uu[2 * w]), den);
-          den = fmaf(__high2float(qq), __uint_as_float(uu[2 * w + 1]), den);
-        }
+        const float den = l_intra + den_inter;
         const int t = c0 + r;
         if (!(den > 0.f) && t < T) flag_status(status, kStatusNonPositiveNormaliser);
-        if (t < T) {
-          const float inv = 1.f / den;
+        const float inv = 1.f / den;                  // rows past T are not stored
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            oo[c] = __float_as_uint(__uint_as_float(oo[c]) * inv);
-            oo2[c] = __float_as_uint(__uint_as_float(oo2[c]) * inv);
-          }
-          uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * T + t) * kDV);
+        for (int c = 0; c < 32; ++c) {
+          oo[c] = __float_as_uint(__uint_as_float(oo[c]) * inv);
+          oo2[c] = __float_as_uint(__uint_as_float(oo2[c]) * inv);
+        }
+        // The stage is free once the previous chunk's store has read it (the
+        // storing thread checks, one chunk late, and tells the others).
+        if (r == 0 && i > 0) {
+          bulk_wait_read_all();
+          mbar_arrive(&bars[kBarStageFree]);
+        }
+        if (i > 0 && !warp_wait(&bars[kBarStageFree], (i - 1) & 1, abort_flag)) break;
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            dst[q4] = pack8(oo + 8 * q4);
-            dst[4 + q4] = pack8(oo2 + 8 * q4);
-          }
+        for (int q4 = 0; q4 < 4; ++q4) {
+          *reinterpret_cast<uint4 *>(stage + sw128(r, q4)) = pack8(oo + 8 * q4);
+          *reinterpret_cast<uint4 *>(stage + sw128(r, 4 + q4)) = pack8(oo2 + 8 * q4);
+        }
+        fence_async_smem();
+        warp_arrive(&bars[kBarStageFull]);
+        if (r == 0 && mbar_wait(&bars[kBarStageFull], i & 1, abort_flag)) {
+          tma_store_3d(&tmo, stage, 0, c0, bh);
+          bulk_commit_group();
         }
       }
+      if (r == 0) bulk_wait_all();                    // stores complete before the CTA exits
     }
   } else if (warp < 10) {
     // -------------------------------------------------- key side (warps 6..9)
@@ -543,6 +628,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     // ---- carry-in: sum of the increments of segments 0 .. g-1 ----
     {
       const float *seg0 = agg + (size_t)bh * G_total * kAggFloats;
+#pragma unroll 1
       for (int m = 0; m < kTiles; ++m) {
         const int f = 128 * m + r;
 #pragma unroll
@@ -575,25 +661,31 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         }
       }
       // Z rows live in lanes 0..31 (quarter 0); the other lanes hold zeros
+      {
+        float acc[32];
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
-        float acc[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+        for (int c = 0; c < 32; ++c) acc[c] = 0.f;
         if (!AGG && r < kDK) {
           for (int gp = 0; gp < g; ++gp) {
-            const float *src = seg0 + (size_t)gp * kAggFloats + kD * kDV + r * kDK + 16 * q2;
+            const float4 *src =
+                reinterpret_cast<const float4 *>(seg0 + (size_t)gp * kAggFloats + kD * kDV + r * kDK);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) acc[c] += src[c];
+            for (int c4 = 0; c4 < 8; ++c4) {
+              const float4 x = src[c4];
+              acc[4 * c4 + 0] += x.x;
+              acc[4 * c4 + 1] += x.y;
+              acc[4 * c4 + 2] += x.z;
+              acc[4 * c4 + 3] += x.w;
+            }
           }
         }
-        uint32_t bits[16];
+        uint32_t bits[32];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) bits[c] = __float_as_uint(acc[c]);
-        tmem_st16(tbase + lane_off + kColZ + 16 * q2, bits);
-        if (!AGG && r < kDK) {
-          *reinterpret_cast<uint4 *>(zsnap + sw64(r, 2 * q2)) = pack8(bits);
-          *reinterpret_cast<uint4 *>(zsnap + sw64(r, 2 * q2 + 1)) = pack8(bits + 8);
+        for (int c = 0; c < 32; ++c) bits[c] = __float_as_uint(acc[c]);
+        tmem_st32(tbase + lane_off + kColZ, bits);
+        if (!AGG && quarter == 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(zsnap + sw64(r, c)) = pack8(bits + 8 * c);
         }
       }
       fence_async_smem();
@@ -609,17 +701,21 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       if (!(ok = warp_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
       // ---- phi(K_c) into the ring, one slot per state tile ----
       {
-        uint32_t XK[16], P[32];
+        uint32_t XK[16], P[32], R2[32];
         load_pairs(smem + L::kOffK + 8192 * st, r, XK, P);
         warp_arrive(&bars[kBarKvEmpty + st]);         // K rows read
 #pragma unroll
+        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[l], 0x40004000u);   // x 2.0
+#pragma unroll 1
         for (int m = 0; m < kTiles; ++m) {
           const int u = i * kTiles + m;
           if (ok) ok = ring_acquire(&bars[kBarKRingEmpty], NK, u);
           if (ok) {
-            write_tile<false>(kring + (u % NK) * kKSlotBytes, r, m, P, P);
+            write_tile(kring + (u % NK) * kKSlotBytes, r, m == kTiles - 1,
+                       m == 0 ? 0x3f003f00u : 0x3f803f80u, P, R2);     // x 1/2 on the diagonal
             ring_publish(&bars[kBarKRingFull], NK, u);
           }
+          rotate_left(R2, 4);
         }
         if (!ok) break;
       }
@@ -673,6 +769,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     const bool write_out = !AGG && g == G_total - 1 && (S_out || z_out);
     if (ok && nchunks > 0 && (write_agg || write_out)) {
       float *dst_agg = agg + ((size_t)bh * G_total + g) * kAggFloats;
+#pragma unroll 1
       for (int m = 0; m < kTiles; ++m) {
         if (m == 4 && quarter != 0) continue;
         const int f = 128 * m + r;
@@ -684,14 +781,16 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
           float *row = write_agg ? dst_agg + (size_t)f * kDV
                                  : (S_out ? S_out + ((size_t)bh * kD + abi_row(f)) * kDV : nullptr);
           if (row) {
+            // increments stay in the internal scaling; S_out is S itself
+            const float sc = (write_agg || f < kDK) ? 1.f : 0.5f;
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
               *reinterpret_cast<float4 *>(row + c) =
-                  make_float4(__uint_as_float(a[c]), __uint_as_float(a[c + 1]),
-                              __uint_as_float(a[c + 2]), __uint_as_float(a[c + 3]));
+                  make_float4(sc * __uint_as_float(a[c]), sc * __uint_as_float(a[c + 1]),
+                              sc * __uint_as_float(a[c + 2]), sc * __uint_as_float(a[c + 3]));
               *reinterpret_cast<float4 *>(row + 32 + c) =
-                  make_float4(__uint_as_float(b2[c]), __uint_as_float(b2[c + 1]),
-                              __uint_as_float(b2[c + 2]), __uint_as_float(b2[c + 3]));
+                  make_float4(sc * __uint_as_float(b2[c]), sc * __uint_as_float(b2[c + 1]),
+                              sc * __uint_as_float(b2[c + 2]), sc * __uint_as_float(b2[c + 3]));
             }
           }
         }
@@ -736,10 +835,11 @@ bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int f
 size_t tc_chunked_agg_floats() { return (size_t)kAggFloats; }
 
 cudaError_t tc_chunked(const ChunkedLaunch &a) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (!make_tma_3d_bf16(&tq, a.q, kDK, a.T, a.BH, kC) ||
       !make_tma_3d_bf16(&tk, a.k, kDK, a.T, a.BH, kC) ||
-      !make_tma_3d_bf16(&tv, a.v, kDV, a.T, a.BH, kC))
+      !make_tma_3d_bf16(&tv, a.v, kDV, a.T, a.BH, kC) ||
+      !make_tma_3d_bf16(&to, a.o, kDV, a.T, a.BH, kC))
     return cudaErrorNotSupported;
   cudaError_t e;
   if (a.G > 1) {
@@ -749,8 +849,7 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
     if (e != cudaSuccess) return e;
     ProfileScope prof("tc_segment_increment", a.stream);
     kagg<<<(unsigned)(a.BH * (a.G - 1)), kThreads, Layout<true>::kSmemBytes, a.stream>>>(
-        tq, tk, tv, static_cast<__nv_bfloat16 *>(a.o), a.agg, nullptr, nullptr, a.status, a.T,
-        a.G - 1, a.G, a.seg_len);
+        tq, tk, tv, to, a.agg, nullptr, nullptr, a.status, a.T, a.G - 1, a.G, a.seg_len);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -760,8 +859,7 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_segment_pass", a.stream);
   kpass<<<(unsigned)(a.BH * a.G), kThreads, Layout<false>::kSmemBytes, a.stream>>>(
-      tq, tk, tv, static_cast<__nv_bfloat16 *>(a.o), a.agg, a.S_out, a.z_out, a.status, a.T, a.G,
-      a.G, a.seg_len);
+      tq, tk, tv, to, a.agg, a.S_out, a.z_out, a.status, a.T, a.G, a.G, a.seg_len);
   return cudaGetLastError();
 }
 
