@@ -24,10 +24,11 @@
 // state is converted to the library's row-major (i <= j) order only where it
 // leaves the kernel (S_out, z_out).
 //
-// Warp roles (352 threads): warp 0 TMA producer; warp 1 TMEM allocation and
-// the query-side MMAs (Q K^T, P V, the readout into O); warp 10 the
-// state-side MMAs (the update of S and Z) - two issuing threads so that one's
-// waits are covered by the other's MMAs; warps 2-5, the query side: the
+// Warp roles (384 threads): warp 0 TMA producer; warp 1 TMEM allocation and
+// the query-side MMAs (Q K^T, P V, U, the even readout slots into O); warp 11
+// the odd readout slots; warp 10 the state-side MMAs (the update of S and Z).
+// Each test of a barrier by an issuing thread stalls its MMA stream, so
+// three issuing threads share the work and cover one another's waits; warps 2-5, the query side: the
 // intra-chunk P, the query features into tensor memory, the epilogue (y
 // staged in shared memory, written by one TMA store per chunk); warps 6-9,
 // the key side: the key features into the shared-memory ring, the bf16
@@ -65,7 +66,7 @@ constexpr int kDK = 32;
 constexpr int kDV = 64;
 constexpr int kD = 528;
 constexpr int kTiles = 5;          // 128-feature state tiles: ceil(528 / 128)
-constexpr int kThreads = 352;      // 11 warps
+constexpr int kThreads = 384;      // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColZ = 320, kColX = 384, kColO = 448;
 constexpr uint32_t kColRing = 352;  // query slot b at kColRing + 32 b (b = 0, 1, 2); U in slot 0
@@ -221,6 +222,17 @@ __device__ __forceinline__ void load_pairs(const uint8_t *tile, int row, uint32_
   }
 }
 
+// Eight fp32 values times inv, rounded to bf16.
+__device__ __forceinline__ uint4 pack8_scaled(const uint32_t *a, float2 inv2) {
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 v = __fmul2_rn(make_float2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1])), inv2);
+    w[j] = tc::pack_bf16x2(v.x, v.y);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 __device__ __forceinline__ uint4 pack8(const uint32_t *a) {
   return make_uint4(tc::pack_bf16x2(__uint_as_float(a[0]), __uint_as_float(a[1])),
                     tc::pack_bf16x2(__uint_as_float(a[2]), __uint_as_float(a[3])),
@@ -267,7 +279,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     mbar_init(&bars[kBarQEmpty], 1 + A);            // Q K^T commit + query side
     for (int st = 0; st < 2; ++st) {
       mbar_init(&bars[kBarKvFull + st], 1);
-      mbar_init(&bars[kBarKvEmpty + st], (AGG ? 1 : 2) + A);   // MMA warp(s) + key side
+      mbar_init(&bars[kBarKvEmpty + st], 2 + A);      // two MMA warps + key side
     }
     mbar_init(&bars[kBarSFull], 1);
     mbar_init(&bars[kBarPFull], A);
@@ -275,15 +287,15 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     mbar_init(&bars[kBarUDone], 1);
     mbar_init(&bars[kBarStageFull], A);
     mbar_init(&bars[kBarStageFree], 1);
-    mbar_init(&bars[kBarOFull], 1);
+    mbar_init(&bars[kBarOFull], 2);                 // both readout issuers
     mbar_init(&bars[kBarXFree], A);
-    mbar_init(&bars[kBarUpdFull], 1);
+    mbar_init(&bars[kBarUpdFull], AGG ? 2 : 1);
     // done-barriers of the snapshots: one commit from each issuing warp (the
     // readout / U that read the old snapshot, the update that wrote the new state)
     mbar_init(&bars[kBarZDone], 2);
     mbar_init(&bars[kBarZSnap], A);
     for (int m = 0; m < 5; ++m) {
-      mbar_init(&bars[kBarTileDone + m], 2);
+      mbar_init(&bars[kBarTileDone + m], 3);       // both readout issuers + the update
       mbar_init(&bars[kBarTileSnap + m], A);
     }
     for (int k = 0; k < kRing; ++k) {
@@ -340,7 +352,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         tma_load_3d(smem + L::kOffV + 16384 * st, &tmv, &bars[kBarKvFull + st], 0, row, bh);
       }
     }
-  } else if (warp == 1 || warp == 10) {
+  } else if (warp == 1 || warp == 10 || warp == 11) {
     // ------------------------------------------------------------ MMA issue
     // Two issuing warps with independent accumulators, so that one's waits
     // are covered by the other's MMAs: warp 1 issues the query side (Q K^T,
@@ -375,8 +387,41 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         return (a || mbar_wait(b1, p1, abort_flag)) && (b || mbar_wait(b2, p2, abort_flag));
       };
       bool ok = true;
+      // O += phi_q(Q) S_c over the readout slots s9 = first, first + 2, ...
+      // (64 features each; slot s9 in ring entry ring_entry(s9), A from tensor
+      // memory, B = rows 64 s9 .. 64 s9 + 63 of the snapshot). Each issuer
+      // releases snapshot tile s9 / 2 after its own slot of that tile.
+      auto readout = [&](int i, int first) -> bool {
+        for (int s9 = first; s9 < kQSlots; s9 += 2) {
+          const int b = ring_entry(s9), k = kRing * i + s9 / kRing;
+          if (!mbar_wait(&bars[kBarRingFull + b], k & 1, abort_flag)) return false;
+          tc_fence_after();
+          const int nk = s9 == kQSlots - 1 ? 1 : 4;
+          const uint32_t a_col = tbase + kColRing + 32 * b;
+          for (int kk = 0; kk < nk; ++kk)
+            mma_ts(tbase + kColO, a_col + 8 * kk, adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
+          mma_commit(&bars[kBarRingEmpty + b]);
+          mma_commit(&bars[kBarTileDone + (s9 >> 1)]);
+        }
+        if (first == 1) mma_commit(&bars[kBarTileDone + (kTiles - 1)]);   // tile 4 has no odd slot
+        return true;
+      };
 
-      if (warp == 1 && !AGG) {
+      if (warp == 11 && !AGG) {
+        // ---------------- odd readout slots; the output store ----------------
+        const uint8_t *stage = smem + L::kOffStage;
+        for (int i = 0; ok && i < nchunks; ++i) {
+          if (!(ok = readout(i, 1))) break;
+          mma_commit(&bars[kBarOFull]);
+          // y of chunk i, staged by the query side, leaves by one TMA store
+          if (!(ok = mbar_wait(&bars[kBarStageFull], i & 1, abort_flag))) break;
+          tma_store_3d(&tmo, stage, 0, t0 + i * kC, bh);
+          bulk_commit_group();
+          bulk_wait_read_all();
+          mbar_arrive(&bars[kBarStageFree]);
+        }
+        bulk_wait_all();                                 // stores complete before the CTA exits
+      } else if (warp == 1 && !AGG) {
         // ---------------- query-side MMAs ----------------
         // Every test of a barrier by an issuing thread drains its MMAs from
         // the tensor pipe, so the issuing threads wait on as few barriers as
@@ -415,34 +460,24 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
           mma_commit(&bars[kBarUDone]);
           mma_commit(&bars[kBarQEmpty]);                 // Q tile no longer read by the tensor core
           mma_commit(&bars[kBarZDone]);                  // Z_c snapshot no longer read
-          // O += phi_q(Q) S_c over nine 64-feature slots (slot s9 in ring
-          // entry ring_entry(s9), A from tensor memory); slots 2m, 2m + 1 read
-          // tile m of the snapshot once it is in place
-          for (int s9 = 0; s9 < kQSlots && ok; ++s9) {
-            const int b = ring_entry(s9), k = kRing * i + s9 / kRing, m = s9 >> 1;
-            if (!(ok = mbar_wait(&bars[kBarRingFull + b], k & 1, abort_flag))) break;
-            tc_fence_after();
-            const int nk = s9 == 8 ? 1 : 4;
-            const uint32_t a_col = tbase + kColRing + 32 * b;
-            for (int kk = 0; kk < nk; ++kk)
-              mma_ts(tbase + kColO, a_col + 8 * kk, adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
-            mma_commit(&bars[kBarRingEmpty + b]);
-            // tile m of the snapshot is no longer read after its last slot
-            if ((s9 & 1) == 1 || s9 == 8) mma_commit(&bars[kBarTileDone + m]);
-          }
-          if (!ok) break;
+          // O += phi_q(Q) S_c over the even readout slots (warp 11 issues
+          // the odd ones)
+          if (!(ok = readout(i, 0))) break;
           mma_commit(&bars[kBarOFull]);
           mma_commit(&bars[kBarKvEmpty + st]);          // this warp's reads of K_i, V_i are done
           if (i + 1 < nchunks && !(ok = issue_qk(i + 1))) break;
         }
-      } else if (warp == 10) {
+      } else if (warp == 10 || (AGG && warp == 1)) {
         // ---------------- state-side MMAs ----------------
+        // In the increment kernel (no readout) warps 10 and 1 split the
+        // tiles (warp 10: Z and tiles 0, 2, 4; warp 1: tiles 1, 3).
         // The key side writes the key features of chunk i after its snapshots
         // of S_i and Z_i (and after K_i, V_i arrived), so a full key-ring slot
         // also says that the state it updates has been read.
         for (int i = 0; ok && i < nchunks; ++i) {
           const int st = i & 1;
           for (int m = 0; m < kTiles && ok; ++m) {
+            if (AGG && (m & 1) != (warp == 1 ? 1 : 0)) continue;
             const int u = i * kTiles + m, b = u % NK;
             if (!(ok = mbar_wait(&bars[kBarKRingFull + b], (u / NK) & 1, abort_flag))) break;
             tc_fence_after();
@@ -481,34 +516,46 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         if (!warp_wait(&bars[kBarSFull], i & 1, abort_flag)) break;
         tc_fence_after();
         // ---- intra-chunk block: P = (Q K^T)^2 masked (key s <= min(r, T-1-c0)) ----
-        // 64 columns per tensor-memory wait; P (bf16) overwrites the columns
-        // already read
+        // 32 keys at a time; P (bf16) overwrites the columns already read.
+        // Per warp, a block of keys is entirely valid, entirely masked (no
+        // load, zeros) or straddles the diagonal (masked per element).
         const int lim = min(r, T - 1 - c0);
+        const int lim_lo = __reduce_min_sync(0xffffffffu, lim);
+        const int lim_hi = __reduce_max_sync(0xffffffffu, lim);
         float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          uint32_t x[2][32];
-          tmem_ld32(tbase + lane_off + kColX + 64 * h, x[0]);
-          tmem_ld32(tbase + lane_off + kColX + 64 * h + 32, x[1]);
-          tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t p[16];
+          if (32 * c > lim_hi) {
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            const int c = 2 * h + c2;
-            uint32_t p[16];
+            for (int k = 0; k < 16; ++k) p[k] = 0u;
+          } else {
+            uint32_t x[32];
+            tmem_ld32(tbase + lane_off + kColX + 32 * c, x);
+            tmem_wait_ld();
+            if (32 * c + 31 <= lim_lo) {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const int s0 = 32 * c + 2 * k;
-              const float2 a =
-                  make_float2(__uint_as_float(x[c2][2 * k]), __uint_as_float(x[c2][2 * k + 1]));
-              float2 w = __fmul2_rn(a, a);
-              w.x = s0 <= lim ? w.x : 0.f;
-              w.y = s0 + 1 <= lim ? w.y : 0.f;
-              lsum[k & 3] = __fadd2_rn(lsum[k & 3], w);
-              p[k] = pack_bf16x2(w.x, w.y);
+              for (int k = 0; k < 16; ++k) {
+                const float2 a = make_float2(__uint_as_float(x[2 * k]), __uint_as_float(x[2 * k + 1]));
+                const float2 w = __fmul2_rn(a, a);
+                lsum[k & 3] = __fadd2_rn(lsum[k & 3], w);
+                p[k] = pack_bf16x2(w.x, w.y);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                const int s0 = 32 * c + 2 * k;
+                const float2 a = make_float2(__uint_as_float(x[2 * k]), __uint_as_float(x[2 * k + 1]));
+                float2 w = __fmul2_rn(a, a);
+                w.x = s0 <= lim ? w.x : 0.f;
+                w.y = s0 + 1 <= lim ? w.y : 0.f;
+                lsum[k & 3] = __fadd2_rn(lsum[k & 3], w);
+                p[k] = pack_bf16x2(w.x, w.y);
+              }
             }
-            tmem_st16(tbase + lane_off + kColX + 16 * c, p);
           }
+          tmem_st16(tbase + lane_off + kColX + 16 * c, p);
         }
         const float2 l01 = __fadd2_rn(lsum[0], lsum[1]), l23 = __fadd2_rn(lsum[2], lsum[3]);
         const float2 lt = __fadd2_rn(l01, l23);
@@ -590,31 +637,17 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int t = c0 + r;
         if (!(den > 0.f) && t < T) flag_status(status, kStatusNonPositiveNormaliser);
         const float inv = 1.f / den;                  // rows past T are not stored
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          oo[c] = __float_as_uint(__uint_as_float(oo[c]) * inv);
-          oo2[c] = __float_as_uint(__uint_as_float(oo2[c]) * inv);
-        }
-        // The stage is free once the previous chunk's store has read it (the
-        // storing thread checks, one chunk late, and tells the others).
-        if (r == 0 && i > 0) {
-          bulk_wait_read_all();
-          mbar_arrive(&bars[kBarStageFree]);
-        }
+        const float2 inv2 = make_float2(inv, inv);
+        // the stage is free once the previous chunk's store has read it
         if (i > 0 && !warp_wait(&bars[kBarStageFree], (i - 1) & 1, abort_flag)) break;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          *reinterpret_cast<uint4 *>(stage + sw128(r, q4)) = pack8(oo + 8 * q4);
-          *reinterpret_cast<uint4 *>(stage + sw128(r, 4 + q4)) = pack8(oo2 + 8 * q4);
+          *reinterpret_cast<uint4 *>(stage + sw128(r, q4)) = pack8_scaled(oo + 8 * q4, inv2);
+          *reinterpret_cast<uint4 *>(stage + sw128(r, 4 + q4)) = pack8_scaled(oo2 + 8 * q4, inv2);
         }
         fence_async_smem();
-        warp_arrive(&bars[kBarStageFull]);
-        if (r == 0 && mbar_wait(&bars[kBarStageFull], i & 1, abort_flag)) {
-          tma_store_3d(&tmo, stage, 0, c0, bh);
-          bulk_commit_group();
-        }
+        warp_arrive(&bars[kBarStageFull]);          // warp 11 stores the tile
       }
-      if (r == 0) bulk_wait_all();                    // stores complete before the CTA exits
     }
   } else if (warp < 10) {
     // -------------------------------------------------- key side (warps 6..9)
