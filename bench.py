@@ -66,25 +66,37 @@ def load_peaks():
             "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
-def source_hash():
+# Source files that define each profiled kernel (a recorded traffic figure is
+# valid only while these are unchanged).
+KERNEL_SOURCES = {
+    "tc_segment_pass": ["chunked_tc.cu", "tc_common.cuh", "common.cuh"],
+    "tc_segment_increment": ["chunked_tc.cu", "tc_common.cuh", "common.cuh"],
+    "tc_quadratic": ["quadratic_tc.cu", "tc_common.cuh", "common.cuh"],
+}
+
+
+def source_hash(kernel=None):
+    """Hash of the kernel's source files (all of csrc when the kernel has no
+    entry in KERNEL_SOURCES)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kernelized_linear_attention_kata_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + f.read())
+    names = KERNEL_SOURCES.get(kernel) or sorted(
+        fn for fn in os.listdir(csrc) if fn.endswith((".cu", ".cuh", ".h")))
+    for fn in sorted(names):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    the current sources of that kernel; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec or rec.get("source_sha") != source_hash():
+    if not rec or rec.get("source_sha") != source_hash(kernel):
         return None
     return rec.get("bytes_per_launch")
 
