@@ -36,6 +36,8 @@ NOMINAL_FP32_TFLOPS_PER_SM_GHZ = 128 * 2 / 1000.0   # 128 FP32 lanes x FMA, per 
 #   hbm: streaming kernel.
 KERNEL_BOUND = {
     "tc_quadratic": "tensor",
+    "tc_fo_pass": "hbm",
+    "tc_fo_increment": "hbm",
     "simt_segment_pass": "alu",
     "simt_segment_increment": "alu",
     "simt_quadratic": "alu",

@@ -97,6 +97,7 @@ struct ChunkedRun {
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
     cudaError_t e = cudaErrorNotSupported;
     if (dtype == KATA_DTYPE_BF16 && tc_chunked_supported(a, DK, DV, a.C, FEAT)) e = tc_chunked(a);
+    else if (dtype == KATA_DTYPE_BF16 && fo_tc_supported(a, DK, DV, a.C, FEAT)) e = fo_tc(a);
     if (e == cudaErrorNotSupported)
       e = dtype == KATA_DTYPE_F32 ? simt_chunked<DK, DV, FEAT, float>(a)
                                   : simt_chunked<DK, DV, FEAT, __nv_bfloat16>(a);

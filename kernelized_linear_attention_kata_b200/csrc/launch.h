@@ -43,6 +43,9 @@ cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature
 bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t tc_chunked(const ChunkedLaunch &a);
 size_t tc_chunked_agg_floats();   // floats of one segment increment
+bool fo_tc_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
+cudaError_t fo_tc(const ChunkedLaunch &a);
+size_t fo_tc_agg_floats();        // floats of one segment increment
 
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_chunked(const ChunkedLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_quadratic(const QuadraticLaunch &a);

@@ -328,3 +328,46 @@ def test_tc_chunked_reports_nonpositive_normaliser():
     q2[0, 0, 300] = 0
     api.kata_fwd_chunked(q2, k, v, o, 128, "psd", workspace=ws)
     assert api.kata_workspace_status(ws) == KATA_ERR_NONPOSITIVE_NORMALISER
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core chunked path, first-order feature (bf16, d_k = d_v = 64)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,H,T,C", [(1, 1, 1, 64), (1, 2, 127, 64), (1, 3, 128, 128), (2, 2, 129, 64),
+                                     (1, 4, 1000, 128), (1, 2, 5000, 64), (2, 40, 300, 64)])
+def test_tc_first_order_shapes_and_state(B, H, T, C):
+    w = W.Workload("tcfo", B=B, H=H, T=T, d_k=64, d_v=64, C=C, dtype="bf16", feature="first_order",
+                   seed=2000 + T + H, recipe="unit")
+    q, k, v = W.make_inputs(w)
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    ref = np.empty((B, H, T, 64))
+    S_ref = np.empty((B, H, 65, 64))
+    z_ref = np.empty((B, H, 65))
+    for b in range(B):
+        for h in range(H):
+            ref[b, h], S_ref[b, h], z_ref[b, h] = O.forward_chunked(
+                qn[b, h], kn[b, h], vn[b, h], C, "first_order", return_state=True)
+    qd, kd, vd = dev(q, k, v)
+    for seq in (False, True):
+        y, S, z = api.fwd_chunked(qd, kd, vd, C, "first_order", return_state=True, sequential=seq)
+        e = rel_err(y.float().cpu().numpy(), ref)
+        assert e <= TOL["bf16"], (seq, e)
+        # the state's products of bf16 inputs are exact; only fp32 summation rounds
+        assert np.max(np.abs(S.cpu().numpy() - S_ref)) <= 1e-4 * np.abs(S_ref).max(), seq
+        assert np.max(np.abs(z.cpu().numpy() - z_ref)) <= 1e-4 * np.abs(z_ref).max(), seq
+
+
+def test_tc_first_order_reports_nonpositive_normaliser():
+    w = W.Workload("tcfoz", B=1, H=1, T=300, d_k=64, d_v=64, C=64, dtype="bf16",
+                   feature="first_order", seed=9, recipe="unit")
+    q, k, v = dev(*W.make_inputs(w))
+    ws = api.alloc_workspace(1, 1, 300, 64, 64, 64, feature="first_order")
+    o = torch.empty_like(v)
+    api.kata_fwd_chunked(q, k, v, o, 64, "first_order", workspace=ws)
+    assert api.kata_workspace_status(ws) == KATA_OK
+    # q_0 = -2 k_0 gives the first token the weight 1 + q.k = -1
+    q2 = q.clone()
+    q2[0, 0, 0] = -2 * k[0, 0, 0]
+    api.kata_fwd_chunked(q2, k, v, o, 64, "first_order", workspace=ws)
+    assert api.kata_workspace_status(ws) == KATA_ERR_NONPOSITIVE_NORMALISER
