@@ -74,6 +74,8 @@ KERNEL_SOURCES = {
     "tc_segment_pass": ["chunked_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_segment_increment": ["chunked_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_quadratic": ["quadratic_tc.cu", "tc_common.cuh", "common.cuh"],
+    "tc_fo_pass": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
+    "tc_fo_increment": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
 }
 
 
