@@ -69,11 +69,16 @@ constexpr int kTiles = 5;          // 128-feature state tiles: ceil(528 / 128)
 constexpr int kThreads = 384;      // 12 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColZ = 320, kColX = 384, kColO = 448;
-constexpr uint32_t kColRing = 352;  // query slot b at kColRing + 32 b (b = 0, 1, 2); U in slot 0
-constexpr int kRing = 3;
-// Ring entry of readout slot s9: entries 1, 2 (P's columns) take the first
-// two slots of a chunk, entry 0 (U's columns) the third, and so on.
-__host__ __device__ constexpr int ring_entry(int s9) { return (s9 + 1) % kRing; }
+constexpr uint32_t kColU = 352;    // U = Q Z_c, then query ring entry 3
+// Query ring: entry 0 is a shared-memory slot (SS readout MMAs), entries 1
+// and 2 are P's columns once P V is done, entry 3 is U's columns once U is
+// read. Readout slot s9 goes to entry s9 mod 4 (entry 0 takes three slots of
+// a chunk, the others two), so warp 1 (even slots) consumes entries 0 and 2
+// and warp 11 (odd slots) entries 1 and 3.
+constexpr int kRing = 4;
+__host__ __device__ constexpr int ring_entry(int s9) { return s9 % kRing; }
+__host__ __device__ constexpr int ring_uses(int e) { return e == 0 ? 3 : 2; }
+__host__ __device__ constexpr uint32_t ring_col(int e) { return e == 3 ? kColU : kColU + 32u * e; }
 constexpr int kAggFloats = kD * kDV + kDK * kDK;      // one segment increment
 
 // Shared memory layout (bytes from a 1024-aligned base). Key features travel
@@ -82,10 +87,11 @@ constexpr int kAggFloats = kD * kDV + kDK * kDK;      // one segment increment
 // slots of 128 token rows x 128 key features, as two 64-feature groups 16 KB
 // apart (update A operand, MN-major), five uses per chunk, one per state tile.
 //   forward pass:  Q 8 KB | K 2 x 8 KB | V 2 x 16 KB | S_c bf16 66 KB |
-//                  Z_c bf16 2 KB | y stage 16 KB | key ring 2 x 32 KB
+//                  Z_c bf16 2 KB | y stage 16 KB | query slot 16 KB | key ring 2 x 32 KB
 //   increments:    K 2 x 8 KB | V 2 x 16 KB | key ring 5 x 32 KB
-// The query features travel through a ring of three tensor-memory slots
-// (readout A operand), nine uses per chunk (64 features each).
+// The query features (readout A operand, 64 features a slot, nine slots a
+// chunk) travel through a ring of one shared-memory slot (128 token rows x
+// 64 features, K-major) and three tensor-memory slots.
 constexpr int kKSlotBytes = 32768;
 constexpr int kQSlots = 9;          // 64-feature readout slots per chunk
 template <bool AGG>
@@ -96,12 +102,13 @@ struct Layout {
   static constexpr int kOffSnap = kOffV + 32768;      // [528][64] bf16, 128 B rows (pass only)
   static constexpr int kOffZSnap = kOffSnap + (AGG ? 0 : kD * 128);   // [32][32] bf16, 64 B rows
   static constexpr int kOffStage = kOffZSnap + (AGG ? 0 : 2048);      // y: [128][64] bf16, 128 B rows
-  static constexpr int kOffKRing = kOffStage + (AGG ? 0 : 16384);
+  static constexpr int kOffQSlot = kOffStage + (AGG ? 0 : 16384);    // query slot (ring entry 0)
+  static constexpr int kOffKRing = kOffQSlot + (AGG ? 0 : 16384);
   static constexpr int kKRingSlots = AGG ? 5 : 2;
   static constexpr int kOffBars = kOffKRing + kKRingSlots * kKSlotBytes;
   static constexpr int kSmemBytes = kOffBars + 1024 + 1024;   // barriers + alignment slack
   static_assert(kOffV % 1024 == 0 && kOffSnap % 1024 == 0 && kOffZSnap % 1024 == 0 &&
-                    kOffStage % 1024 == 0 && kOffKRing % 1024 == 0,
+                    kOffStage % 1024 == 0 && kOffQSlot % 1024 == 0 && kOffKRing % 1024 == 0,
                 "swizzle atoms need 1024-byte alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -388,18 +395,25 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       };
       bool ok = true;
       // O += phi_q(Q) S_c over the readout slots s9 = first, first + 2, ...
-      // (64 features each; slot s9 in ring entry ring_entry(s9), A from tensor
-      // memory, B = rows 64 s9 .. 64 s9 + 63 of the snapshot). Each issuer
-      // releases snapshot tile s9 / 2 after its own slot of that tile.
+      // (64 features each; slot s9 in ring entry ring_entry(s9), A from the
+      // shared-memory slot or tensor memory, B = rows 64 s9 .. 64 s9 + 63 of
+      // the snapshot). Each issuer releases snapshot tile s9 / 2 after its own
+      // slot of that tile.
+      const uint64_t d_qslot = smem_desc(smem_u32(smem + L::kOffQSlot), 16, 1024, kSw128);
       auto readout = [&](int i, int first) -> bool {
         for (int s9 = first; s9 < kQSlots; s9 += 2) {
-          const int b = ring_entry(s9), k = kRing * i + s9 / kRing;
+          const int b = ring_entry(s9), k = ring_uses(b) * i + s9 / kRing;
           if (!mbar_wait(&bars[kBarRingFull + b], k & 1, abort_flag)) return false;
           tc_fence_after();
           const int nk = s9 == kQSlots - 1 ? 1 : 4;
-          const uint32_t a_col = tbase + kColRing + 32 * b;
-          for (int kk = 0; kk < nk; ++kk)
-            mma_ts(tbase + kColO, a_col + 8 * kk, adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
+          if (b == 0) {
+            for (int kk = 0; kk < nk; ++kk)
+              mma_ss(tbase + kColO, adv(d_qslot, 32 * kk), adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
+          } else {
+            const uint32_t a_col = tbase + ring_col(b);
+            for (int kk = 0; kk < nk; ++kk)
+              mma_ts(tbase + kColO, a_col + 8 * kk, adv(d_snap, (64 * s9 + 16 * kk) * 128), id_ro, 1);
+          }
           mma_commit(&bars[kBarRingEmpty + b]);
           mma_commit(&bars[kBarTileDone + (s9 >> 1)]);
         }
@@ -456,7 +470,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
           // U = Q Z_c into query slot 0
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_ss(tbase + kColRing, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_u, kk);
+            mma_ss(tbase + kColU, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_u, kk);
           mma_commit(&bars[kBarUDone]);
           mma_commit(&bars[kBarQEmpty]);                 // Q tile no longer read by the tensor core
           mma_commit(&bars[kBarZDone]);                  // Z_c snapshot no longer read
@@ -510,6 +524,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       const int r = quarter * 32 + lane;                  // TMEM lane = token of the chunk
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
       uint8_t *stage = smem + L::kOffStage;
+      uint8_t *qslot = smem + L::kOffQSlot;
       for (int i = 0; i < nchunks; ++i) {
         const int c0 = t0 + i * kC;
         if (!warp_wait(&bars[kBarQFull], i & 1, abort_flag)) break;
@@ -577,21 +592,23 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         for (int l = 0; l < 32; ++l) R[l] = P[l];
 #pragma unroll 1
         for (int s9 = 0; s9 < kQSlots; ++s9) {
-          const int b = ring_entry(s9), j = s9 / kRing, k = kRing * i + j;
+          const int b = ring_entry(s9), j = s9 / kRing, k = ring_uses(b) * i + j;
           // Entry b may be written once its previous use has been read. The
-          // first use of a chunk instead waits for what last used the columns
-          // in this chunk (P V for entries 1 and 2, U for entry 0), which
-          // also implies every use of the previous chunk is complete; entry 0
-          // first hands its U to the denominator.
+          // first use of a chunk of a tensor-memory entry instead waits for
+          // what last used the columns in this chunk (P V for entries 1 and
+          // 2, U for entry 3), which also implies every use of the previous
+          // chunk is complete; entry 3 first hands its U to the denominator.
           if (ok) {
             if (j == 0 && b == 1) {
               ok = warp_wait(&bars[kBarPVDone], i & 1, abort_flag);
-            } else if (j == 0 && b == 0) {
+            } else if (j == 0 && b == 2) {
+              // P V already waited for (entry 1 comes first)
+            } else if (j == 0 && b == 3) {
               ok = warp_wait(&bars[kBarUDone], i & 1, abort_flag);
               if (ok) {
                 tc_fence_after();
                 uint32_t uu[32];
-                tmem_ld32(tbase + lane_off + kColRing, uu);
+                tmem_ld32(tbase + lane_off + kColU, uu);
                 tmem_wait_ld();
 #pragma unroll
                 for (int w = 0; w < 16; ++w) {
@@ -600,7 +617,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                   den_inter = fmaf(__high2float(qq), __uint_as_float(uu[2 * w + 1]), den_inter);
                 }
               }
-            } else if (j > 0) {
+            } else if (k > 0) {
               ok = warp_wait(&bars[kBarRingEmpty + b], (k - 1) & 1, abort_flag);
             }
           }
@@ -610,9 +627,17 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             tc_fence_after();
             uint32_t w[32];
             q_slot_words(P, R, s9 == kQSlots - 1, w);
-            tmem_st32(tbase + lane_off + kColRing + 32 * b, w);
-            tmem_wait_st();
-            tc_fence_before();
+            if (b == 0) {
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc)
+                *reinterpret_cast<uint4 *>(qslot + sw128(r, cc)) =
+                    make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+              fence_async_smem();
+            } else {
+              tmem_st32(tbase + lane_off + ring_col(b), w);
+              tmem_wait_st();
+              tc_fence_before();
+            }
             warp_arrive(&bars[kBarRingFull + b]);
           }
           rotate_left(R, 2);
