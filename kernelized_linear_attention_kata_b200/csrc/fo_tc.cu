@@ -47,11 +47,12 @@ constexpr int kThreads = 320;      // 10 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 128, kColX = 256;   // X of tile i at kColX + 128 (i & 1)
 constexpr int kAggFloats = kRows * kRows;                 // one segment increment: S'[0..64][0..64]
+constexpr int kStages = 3;                                // Q, K, V tiles in flight
 
 // Shared memory (bytes from a 1024-aligned base):
-//   pass: Q 2 x 16 KB | K 2 x 16 KB | V 2 x 16 KB | ones 16 KB | ones(A) 4 KB |
+//   pass: Q 3 x 16 KB | K 3 x 16 KB | V 3 x 16 KB | ones 16 KB | ones(A) 4 KB |
 //         S' snapshot 2 x 10 KB | y stage 16 KB
-//   increments: K 2 x 16 KB | V 2 x 16 KB | ones 16 KB
+//   increments: K 3 x 16 KB | V 3 x 16 KB | ones 16 KB
 // "ones": 128 rows of 128 B whose element 0 is 1 (SW128): the second
 // 64-element group of the MN-major operands [K | 1]^T (feature 64 = the
 // constant) and [V | 1] (column 64 = the count). "ones(A)": 128 rows of 32 B
@@ -59,9 +60,9 @@ constexpr int kAggFloats = kRows * kRows;                 // one segment increme
 template <bool AGG>
 struct FoLayout {
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = AGG ? 0 : 32768;
-  static constexpr int kOffV = kOffK + 32768;
-  static constexpr int kOffOnes = kOffV + 32768;
+  static constexpr int kOffK = AGG ? 0 : kStages * 16384;
+  static constexpr int kOffV = kOffK + kStages * 16384;
+  static constexpr int kOffOnes = kOffV + kStages * 16384;
   static constexpr int kOffOnesA = kOffOnes + 16384;
   static constexpr int kOffSnap = kOffOnesA + (AGG ? 0 : 4096);
   static constexpr int kSnapGroup = kNa * 128;                // 10 KB per 64-column group
@@ -74,7 +75,8 @@ struct FoLayout {
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 enum {
-  kBarQFull = 0, kBarQEmpty = 2, kBarKvFull = 4, kBarKvEmpty = 6, kBarSFull = 8, kBarPFull = 10,
+  kBarQFull = 0, kBarQEmpty = kBarQFull + kStages, kBarKvFull = kBarQEmpty + kStages,
+  kBarKvEmpty = kBarKvFull + kStages, kBarSFull = kBarKvEmpty + kStages, kBarPFull = kBarSFull + 2,
   kBarOFull, kBarSnapFull, kBarSnapFree, kBarStageFull, kBarStageFree, kBarUpdFull, kNumBars
 };
 constexpr int kBarBytes = 8 * kNumBars;
@@ -147,13 +149,13 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
   fence_async_smem();
   if (threadIdx.x == 0) {
     constexpr uint32_t A = kSetArrivals;
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars[kBarQFull + s], 1);
       mbar_init(&bars[kBarQEmpty + s], 1);
       mbar_init(&bars[kBarKvFull + s], 1);
       mbar_init(&bars[kBarKvEmpty + s], 1);
-      mbar_init(&bars[kBarSFull + s], 1);
     }
+    for (int s = 0; s < 2; ++s) mbar_init(&bars[kBarSFull + s], 1);
     mbar_init(&bars[kBarPFull], A);
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarSnapFull], A);
@@ -180,14 +182,14 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       tma_prefetch_desc(&tmv);
       if (!AGG) tma_prefetch_desc(&tmq);
       for (int i = 0; i < ntiles; ++i) {
-        const int st = i & 1, row = t0 + i * kTile;
-        const uint32_t par = ((i >> 1) - 1) & 1;
+        const int st = i % kStages, row = t0 + i * kTile;
+        const uint32_t par = ((i / kStages) - 1) & 1;
         if (!AGG) {
-          if (i >= 2 && !mbar_wait(&bars[kBarQEmpty + st], par, abort_flag)) break;
+          if (i >= kStages && !mbar_wait(&bars[kBarQEmpty + st], par, abort_flag)) break;
           mbar_arrive_expect_tx(&bars[kBarQFull + st], 16384);
           tma_load_3d(smem + L::kOffQ + 16384 * st, &tmq, &bars[kBarQFull + st], 0, row, bh);
         }
-        if (i >= 2 && !mbar_wait(&bars[kBarKvEmpty + st], par, abort_flag)) break;
+        if (i >= kStages && !mbar_wait(&bars[kBarKvEmpty + st], par, abort_flag)) break;
         mbar_arrive_expect_tx(&bars[kBarKvFull + st], 32768);
         tma_load_3d(smem + L::kOffK + 16384 * st, &tmk, &bars[kBarKvFull + st], 0, row, bh);
         tma_load_3d(smem + L::kOffV + 16384 * st, &tmv, &bars[kBarKvFull + st], 0, row, bh);
@@ -204,8 +206,8 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       const uint32_t a_q = smem_u32(smem + L::kOffQ), a_k = smem_u32(smem + L::kOffK);
       const uint32_t a_v = smem_u32(smem + L::kOffV), a_ones = smem_u32(smem + L::kOffOnes);
       // [V | 1] and [K | 1]^T, MN-major: the second 64-element group is the ones tile
-      uint64_t d_v1[2], d_k1[2], d_kk[2], d_q[2];
-      for (int s = 0; s < 2; ++s) {
+      uint64_t d_v1[kStages], d_k1[kStages], d_kk[kStages], d_q[kStages];
+      for (int s = 0; s < kStages; ++s) {
         d_v1[s] = smem_desc(a_v + 16384 * s, a_ones - (a_v + 16384 * s), 1024, kSw128);
         d_k1[s] = smem_desc(a_k + 16384 * s, a_ones - (a_k + 16384 * s), 1024, kSw128);
         d_kk[s] = smem_desc(a_k + 16384 * s, 16, 1024, kSw128);     // K, K-major (Q K^T's B)
@@ -216,8 +218,8 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       bool ok = true;
       if (AGG) {
         for (int i = 0; ok && i < ntiles; ++i) {
-          const int st = i & 1;
-          if (!(ok = mbar_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
+          const int st = i % kStages;
+          if (!(ok = mbar_wait(&bars[kBarKvFull + st], (i / kStages) & 1, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -228,11 +230,11 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         if (ok && ntiles > 0) mma_commit(&bars[kBarUpdFull]);
       } else {
         auto issue_qk = [&](int i) {
-          const int st = i & 1;
+          const int st = i % kStages, xb = i & 1;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tbase + kColX + 128 * st, adv(d_q[st], 32 * kk), adv(d_kk[st], 32 * kk), id_qk, kk);
-          mma_commit(&bars[kBarSFull + st]);
+            mma_ss(tbase + kColX + 128 * xb, adv(d_q[st], 32 * kk), adv(d_kk[st], 32 * kk), id_qk, kk);
+          mma_commit(&bars[kBarSFull + xb]);
         };
         if (ntiles > 0) {
           ok = mbar_wait(&bars[kBarQFull], 0, abort_flag) && mbar_wait(&bars[kBarKvFull], 0, abort_flag);
@@ -244,12 +246,12 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         // PFull(i) also says: the snapshot of S'_i is in place, tile i + 1's
         // Q, K, V are loaded, and O' was read by the previous epilogue.
         for (int i = 0; ok && i < ntiles; ++i) {
-          const int st = i & 1;
+          const int st = i % kStages;
           if (!(ok = mbar_wait(&bars[kBarPFull], i & 1, abort_flag))) break;
           tc_fence_after();
           if (i + 1 < ntiles) issue_qk(i + 1);
           // O' = P [V | 1]  (P from tensor memory)
-          const uint32_t x = tbase + kColX + 128 * st;
+          const uint32_t x = tbase + kColX + 128 * (i & 1);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tbase + kColO, x + 8 * kk, adv(d_v1[st], 2048 * kk), id_pv, kk);
@@ -277,11 +279,11 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
       uint8_t *stage = smem + L::kOffStage;
       for (int i = 0; i < ntiles; ++i) {
-        const int st = i & 1, c0 = t0 + i * kTile;
-        if (!warp_wait(&bars[kBarSFull + st], (i >> 1) & 1, abort_flag)) break;
+        const int xb = i & 1, c0 = t0 + i * kTile;
+        if (!warp_wait(&bars[kBarSFull + xb], (i >> 1) & 1, abort_flag)) break;
         tc_fence_after();
         // ---- P = (1 + Q K^T) masked to keys s <= min(r, t1 - 1 - c0) ----
-        const uint32_t x = tbase + lane_off + kColX + 128 * st;
+        const uint32_t x = tbase + lane_off + kColX + 128 * xb;
         const int lim = min(r, t1 - 1 - c0);
         const int lim_lo = __reduce_min_sync(0xffffffffu, lim);
         const int lim_hi = __reduce_max_sync(0xffffffffu, lim);
@@ -313,9 +315,11 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         tc_fence_before();
         // fold the MMA warp's other dependencies into PFull
         bool ok = warp_wait(&bars[kBarSnapFull], i & 1, abort_flag);
-        if (ok && i + 1 < ntiles)
-          ok = warp_wait(&bars[kBarQFull + (st ^ 1)], ((i + 1) >> 1) & 1, abort_flag) &&
-               warp_wait(&bars[kBarKvFull + (st ^ 1)], ((i + 1) >> 1) & 1, abort_flag);
+        if (ok && i + 1 < ntiles) {
+          const int sn = (i + 1) % kStages;
+          const uint32_t pn = ((i + 1) / kStages) & 1;
+          ok = warp_wait(&bars[kBarQFull + sn], pn, abort_flag) && warp_wait(&bars[kBarKvFull + sn], pn, abort_flag);
+        }
         if (!ok) break;
         mbar_arrive(&bars[kBarPFull]);
 
