@@ -235,6 +235,25 @@ def run_reference(args, rank, world):
     return 0
 
 
+def max_over_ranks(x, world, device):
+    """The largest x of all ranks (every rank gets it): a multi-GPU time is
+    the slowest rank's."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(ms_per_step, tokens_per_step, world, device):
+    """Whole-job tokens/s of `world` replicas, each processing tokens_per_step
+    per step: all ranks' tokens over the slowest rank's step time."""
+    ms = max_over_ranks(ms_per_step, world, device)
+    return world * tokens_per_step / (ms / 1e3), ms
+
+
 def workload_config(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_k": w.d_k, "d_v": w.d_v,
             "C": w.C, "feature": w.feature, "form": "chunked (segmented scan carry)",
@@ -336,11 +355,7 @@ def run_ours(args, rank, world, local_rank):
         prof = api.profile_read()
         api.profile_enable(False)
     ms = start.elapsed_time(end) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * tokens_per_step / (ms / 1e3)
+    value, ms = aggregate_throughput(ms, tokens_per_step, world, dev)
 
     # roofline of the dominant kernel, timed live by the library's events
     peaks = load_peaks()
@@ -401,11 +416,8 @@ def run_ours(args, rank, world, local_rank):
         e2.record(stream)
         torch.cuda.synchronize()
         ms_e2e = s2.elapsed_time(e2) / n_e2e
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": world * tokens_per_step / (ms_e2e / 1e3), "unit": UNIT,
+        e2e_value, ms_e2e = aggregate_throughput(ms_e2e, tokens_per_step, world, dev)
+        e2e = {"value": e2e_value, "unit": UNIT,
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (q, k, v)),
                "d2h_bytes_per_step": o.numel() * o.element_size(), "ms_per_step": ms_e2e}
 
