@@ -163,30 +163,43 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const int row = quarter * 32 + lane;
     const int t = qb * kBlock + row;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float l = 0.f;
+    // row sum of the weights in four packed partial sums (no long add chain)
+    float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
     bool ok = true;
     for (int j = 0; j < nkb; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int key0 = j * kBlock;
-#pragma unroll
+      // key blocks below the diagonal block lie entirely before every query
+      // of this block (and before T): no mask there
+      const bool diag = j == nkb - 1;
+#pragma unroll 1
       for (int c = 0; c < kBlock / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tbase + lane_off + kColS + 32 * c, r);
         tmem_wait_ld();
         uint32_t p[16];
+        if (!diag) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k0 = key0 + 32 * c + 2 * i;
-          const float x0 = __uint_as_float(r[2 * i]);
-          const float x1 = __uint_as_float(r[2 * i + 1]);
-          float w0 = FEAT == kPSD ? x0 * x0 : 1.f + x0;
-          float w1 = FEAT == kPSD ? x1 * x1 : 1.f + x1;
-          if (k0 > t || k0 >= T) w0 = 0.f;
-          if (k0 + 1 > t || k0 + 1 >= T) w1 = 0.f;
-          l += w0 + w1;
-          p[i] = pack_bf16x2(w0, w1);
+          for (int i = 0; i < 16; ++i) {
+            const float2 x = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            const float2 w = FEAT == kPSD ? __fmul2_rn(x, x) : __fadd2_rn(make_float2(1.f, 1.f), x);
+            lsum[i & 3] = __fadd2_rn(lsum[i & 3], w);
+            p[i] = pack_bf16x2(w.x, w.y);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int k0 = key0 + 32 * c + 2 * i;
+            const float2 x = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            float2 w = FEAT == kPSD ? __fmul2_rn(x, x) : __fadd2_rn(make_float2(1.f, 1.f), x);
+            if (k0 > t || k0 >= T) w.x = 0.f;
+            if (k0 + 1 > t || k0 + 1 >= T) w.y = 0.f;
+            lsum[i & 3] = __fadd2_rn(lsum[i & 3], w);
+            p[i] = pack_bf16x2(w.x, w.y);
+          }
         }
         tmem_st16(tbase + lane_off + kColS + 16 * c, p);
       }
@@ -194,6 +207,8 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       tc_fence_before();
       mbar_arrive(p_full);
     }
+    const float2 l01 = __fadd2_rn(lsum[0], lsum[1]), l23 = __fadd2_rn(lsum[2], lsum[3]);
+    const float l = (l01.x + l01.y) + (l23.x + l23.y);
     // warp-uniform: the TMEM loads below are warp-collective
     const bool have_o = __all_sync(0xffffffffu, ok && mbar_wait(o_full, 0, abort_flag));
     if (have_o) tc_fence_after();
