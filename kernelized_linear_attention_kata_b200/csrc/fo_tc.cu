@@ -20,10 +20,12 @@
 // segment's increment of S', the second gives segment g the sum of the
 // increments of segments 0 .. g-1 as its carry-in.
 //
-// Warp roles (320 threads): warp 0 TMA (Q, K, V, two stages each); warp 1
-// TMEM allocation and every MMA; warps 2-5 the query side (P, the epilogue);
-// warps 6-9 the state side (the bf16 snapshot of S' after each update, the
-// carry-in, the state written out, the TMA store of y). Math thread r owns
+// Warp roles (320 threads): warp 0 TMA (Q, K, V, three stages each); warp 1
+// TMEM allocation and every MMA; warps 2-5 the query side (P); warps 6-9 the
+// state side (the bf16 snapshot of S' after each update, the epilogue and
+// the TMA store of y, the carry-in, the state written out). Per tile the
+// MMA warp issues the update before the readout, so the snapshot of S'_i+1
+// (double-buffered) is taken while the readout of tile i runs. Math thread r owns
 // TMEM lane r: token r of the tile, or feature row r of S'.
 //
 // Tensor memory (512 columns): S' [0, 80) (lanes 0..64 used), O' [128, 208),
@@ -51,7 +53,7 @@ constexpr int kStages = 3;                                // Q, K, V tiles in fl
 
 // Shared memory (bytes from a 1024-aligned base):
 //   pass: Q 3 x 16 KB | K 3 x 16 KB | V 3 x 16 KB | ones 16 KB | ones(A) 4 KB |
-//         S' snapshot 2 x 10 KB | y stage 16 KB
+//         S' snapshots 2 x (2 x 10 KB) | y stage 16 KB
 //   increments: K 3 x 16 KB | V 3 x 16 KB | ones 16 KB
 // "ones": 128 rows of 128 B whose element 0 is 1 (SW128): the second
 // 64-element group of the MN-major operands [K | 1]^T (feature 64 = the
@@ -66,7 +68,8 @@ struct FoLayout {
   static constexpr int kOffOnesA = kOffOnes + 16384;
   static constexpr int kOffSnap = kOffOnesA + (AGG ? 0 : 4096);
   static constexpr int kSnapGroup = kNa * 128;                // 10 KB per 64-column group
-  static constexpr int kOffStage = kOffSnap + (AGG ? 0 : 2 * kSnapGroup);
+  static constexpr int kSnapBytes = 2 * kSnapGroup;            // one snapshot (two groups)
+  static constexpr int kOffStage = kOffSnap + (AGG ? 0 : 2 * kSnapBytes);   // two snapshots
   static constexpr int kOffBars = kOffStage + (AGG ? 0 : 16384);
   static constexpr int kSmemBytes = kOffBars + 1024 + 1024;
   static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffOnes % 1024 == 0 &&
@@ -77,7 +80,7 @@ struct FoLayout {
 enum {
   kBarQFull = 0, kBarQEmpty = kBarQFull + kStages, kBarKvFull = kBarQEmpty + kStages,
   kBarKvEmpty = kBarKvFull + kStages, kBarSFull = kBarKvEmpty + kStages, kBarPFull = kBarSFull + 2,
-  kBarOFull, kBarSnapFull, kBarSnapFree, kBarStageFull, kBarStageFree, kBarUpdFull, kNumBars
+  kBarOFull, kBarOFree, kBarSnapFull, kBarSnapFree, kBarStageFull, kBarStageFree, kBarUpdFull, kNumBars
 };
 constexpr int kBarBytes = 8 * kNumBars;
 
@@ -143,7 +146,7 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       *reinterpret_cast<uint4 *>(smem + L::kOffOnesA + i * 16) = v;
     }
     // snapshot rows 65..79 and the unused chunks of the second group stay zero
-    for (int i = threadIdx.x; i < 2 * L::kSnapGroup / 16; i += kThreads)
+    for (int i = threadIdx.x; i < 2 * L::kSnapBytes / 16; i += kThreads)
       *reinterpret_cast<uint4 *>(smem + L::kOffSnap + i * 16) = make_uint4(0u, 0u, 0u, 0u);
   }
   fence_async_smem();
@@ -158,6 +161,7 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
     for (int s = 0; s < 2; ++s) mbar_init(&bars[kBarSFull + s], 1);
     mbar_init(&bars[kBarPFull], A);
     mbar_init(&bars[kBarOFull], 1);
+    mbar_init(&bars[kBarOFree], A);
     mbar_init(&bars[kBarSnapFull], A);
     mbar_init(&bars[kBarSnapFree], 1);
     mbar_init(&bars[kBarStageFull], A);
@@ -255,18 +259,23 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tbase + kColO, x + 8 * kk, adv(d_v1[st], 2048 * kk), id_pv, kk);
-          // O' += [Q | 1] S'_i
-#pragma unroll
-          for (int kk = 0; kk < 5; ++kk)
-            mma_ss(tbase + kColO, kk < 4 ? adv(d_q[st], 32 * kk) : d_q1, adv(d_snap, 2048 * kk), id_ro, 1);
-          mma_commit(&bars[kBarOFull]);
-          mma_commit(&bars[kBarQEmpty + st]);
-          // S' += [K | 1]^T [V | 1]
+          // S' += [K | 1]^T [V | 1] first: the readout below reads the
+          // snapshot of S'_i (in shared memory), so the state side can take
+          // the snapshot of S'_i+1 while the readout runs
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(tbase + kColS, adv(d_k1[st], 2048 * kk), adv(d_v1[st], 2048 * kk), id_up, 1);
-          mma_commit(&bars[kBarSnapFree]);                // snapshot read, S' updated
+          // S' updated; also tile i - 1's readout (issued before) has read
+          // the other snapshot buffer
+          mma_commit(&bars[kBarSnapFree]);
           mma_commit(&bars[kBarKvEmpty + st]);
+          // O' += [Q | 1] S'_i
+          const uint64_t d_sn = adv(d_snap, (i & 1) * L::kSnapBytes);
+#pragma unroll
+          for (int kk = 0; kk < 5; ++kk)
+            mma_ss(tbase + kColO, kk < 4 ? adv(d_q[st], 32 * kk) : d_q1, adv(d_sn, 2048 * kk), id_ro, 1);
+          mma_commit(&bars[kBarOFull]);
+          mma_commit(&bars[kBarQEmpty + st]);
         }
         if (ok && ntiles > 0) mma_commit(&bars[kBarUpdFull]);
       }
@@ -277,7 +286,6 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       const int quarter = warp & 3;
       const int r = quarter * 32 + lane;
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      uint8_t *stage = smem + L::kOffStage;
       for (int i = 0; i < ntiles; ++i) {
         const int xb = i & 1, c0 = t0 + i * kTile;
         if (!warp_wait(&bars[kBarSFull + xb], (i >> 1) & 1, abort_flag)) break;
@@ -313,8 +321,10 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         }
         tmem_wait_st();
         tc_fence_before();
-        // fold the MMA warp's other dependencies into PFull
+        // fold the MMA warp's other dependencies into PFull: the snapshot of
+        // S'_i, O' read by the previous epilogue, tile i + 1's Q, K, V
         bool ok = warp_wait(&bars[kBarSnapFull], i & 1, abort_flag);
+        if (ok && i > 0) ok = warp_wait(&bars[kBarOFree], (i - 1) & 1, abort_flag);
         if (ok && i + 1 < ntiles) {
           const int sn = (i + 1) % kStages;
           const uint32_t pn = ((i + 1) / kStages) & 1;
@@ -322,28 +332,6 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
         }
         if (!ok) break;
         mbar_arrive(&bars[kBarPFull]);
-
-        // ---- epilogue: y = O'[:, 0:64] / O'[:, 64] ----
-        if (!warp_wait(&bars[kBarOFull], i & 1, abort_flag)) break;
-        tc_fence_after();
-        uint32_t oa[32], ob[32], oc[16];
-        tmem_ld32(tbase + lane_off + kColO, oa);
-        tmem_ld32(tbase + lane_off + kColO + 32, ob);
-        tmem_ld16(tbase + lane_off + kColO + 64, oc);
-        tmem_wait_ld();
-        tc_fence_before();
-        const float den = __uint_as_float(oc[0]);
-        if (!(den > 0.f) && c0 + r < t1) flag_status(status, kStatusNonPositiveNormaliser);
-        const float inv = 1.f / den;                    // rows past the segment are not stored
-        const float2 inv2 = make_float2(inv, inv);
-        if (i > 0 && !warp_wait(&bars[kBarStageFree], (i - 1) & 1, abort_flag)) break;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          *reinterpret_cast<uint4 *>(stage + sw128(r, q4)) = pack8_scaled(oa + 8 * q4, inv2);
-          *reinterpret_cast<uint4 *>(stage + sw128(r, 4 + q4)) = pack8_scaled(ob + 8 * q4, inv2);
-        }
-        fence_async_smem();
-        mbar_arrive(&bars[kBarStageFull]);
       }
     }
   } else {
@@ -355,8 +343,9 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
     const bool rows = quarter < 3;                      // warps holding rows 0..64 (row 64 in quarter 2)
     bool ok = true;
     // snapshot of S' rows 0..64 (80 columns) as the readout's bf16 B operand
-    auto snapshot = [&]() {
+    auto snapshot = [&](int buf) {
       if (!rows) return;
+      uint8_t *sn = snap + buf * L::kSnapBytes;
       uint32_t a[32], b[32], c[16];
       tmem_ld32(tbase + lane_off + kColS, a);
       tmem_ld32(tbase + lane_off + kColS + 32, b);
@@ -365,12 +354,12 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       if (r < kRows) {
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          *reinterpret_cast<uint4 *>(snap + sw128(r, q4)) = pack8(a + 8 * q4);
-          *reinterpret_cast<uint4 *>(snap + sw128(r, 4 + q4)) = pack8(b + 8 * q4);
+          *reinterpret_cast<uint4 *>(sn + sw128(r, q4)) = pack8(a + 8 * q4);
+          *reinterpret_cast<uint4 *>(sn + sw128(r, 4 + q4)) = pack8(b + 8 * q4);
         }
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2)
-          *reinterpret_cast<uint4 *>(snap + L::kSnapGroup + sw128(r, q2)) = pack8(c + 8 * q2);
+          *reinterpret_cast<uint4 *>(sn + L::kSnapGroup + sw128(r, q2)) = pack8(c + 8 * q2);
       }
     };
 
@@ -393,23 +382,47 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       tmem_st32(tbase + lane_off + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(bits + 32));
       tmem_st16(tbase + lane_off + kColS + 64, *reinterpret_cast<uint32_t(*)[16]>(bits + 64));
       tmem_wait_st();
-      snapshot();
+      snapshot(0);
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[kBarSnapFull]);
     }
 
-    const uint8_t *stage = smem + L::kOffStage;
+    uint8_t *stage = smem + L::kOffStage;
     for (int i = 0; !AGG && ok && i < ntiles; ++i) {
-      // snapshot of S'_i+1 once tile i's readout and update are done
+      const int c0 = t0 + i * kTile;
+      // snapshot of S'_i+1 (into buffer (i + 1) & 1) once tile i's update is
+      // done, which also means tile i - 1's readout has read that buffer
       if (i + 1 < ntiles) {
         if (!(ok = warp_wait(&bars[kBarSnapFree], i & 1, abort_flag))) break;
         tc_fence_after();
-        snapshot();
+        snapshot((i + 1) & 1);
         fence_async_smem();
         tc_fence_before();
         mbar_arrive(&bars[kBarSnapFull]);
       }
+      // ---- epilogue: y = O'[:, 0:64] / O'[:, 64] (row r = token r) ----
+      if (!(ok = warp_wait(&bars[kBarOFull], i & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t oa[32], ob[32], oc[16];
+      tmem_ld32(tbase + lane_off + kColO, oa);
+      tmem_ld32(tbase + lane_off + kColO + 32, ob);
+      tmem_ld16(tbase + lane_off + kColO + 64, oc);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars[kBarOFree]);                   // O' may be overwritten
+      const float den = __uint_as_float(oc[0]);
+      if (!(den > 0.f) && c0 + r < t1) flag_status(status, kStatusNonPositiveNormaliser);
+      const float inv = 1.f / den;                      // rows past the segment are not stored
+      const float2 inv2 = make_float2(inv, inv);
+      if (i > 0 && !(ok = warp_wait(&bars[kBarStageFree], (i - 1) & 1, abort_flag))) break;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        *reinterpret_cast<uint4 *>(stage + sw128(r, q4)) = pack8_scaled(oa + 8 * q4, inv2);
+        *reinterpret_cast<uint4 *>(stage + sw128(r, 4 + q4)) = pack8_scaled(ob + 8 * q4, inv2);
+      }
+      fence_async_smem();
+      mbar_arrive(&bars[kBarStageFull]);
       // y of tile i leaves by one TMA store (one thread)
       if (r == 0) {
         ok = mbar_wait(&bars[kBarStageFull], i & 1, abort_flag);
