@@ -14,6 +14,10 @@ Parity status per function (what pins it is listed in tests/test_oracle_pins.py)
                                          -- pinned against the brute force and
   against each other on tiny inputs, plus the same closed forms.
 * exclusive_tree_scan                    -- pinned against a running sum.
+* backward_brute_force, backward_rows (oracle/backward.py)
+                                         -- pinned by central finite
+  differences of forward_brute_force and by closed forms (T = 1, the
+  normalisation identity, PSD homogeneity, equal keys, q = 0).
 * the first-order feature phi_1(u) = [1, u] -- the arithmetic is pinned (hand
   fixture, forms agreement), but the READING that this is the pages'
   "first-order feature" is not fixed by the pages: parity of that reading is
@@ -28,3 +32,4 @@ from .kata import (  # noqa: F401
     forward_recurrent_unpacked, forward_rows, key_feature, per_head, psd_key_feature,
     psd_pairs, psd_query_feature, query_feature, state_dim, weights,
 )
+from .backward import backward_brute_force, backward_rows  # noqa: F401
