@@ -42,7 +42,12 @@ KERNEL_BOUND = {
     "simt_segment_increment": "alu",
     "simt_quadratic": "alu",
     "simt_decode": "hbm",
+    "simt_bwd_dq": "alu",
+    "simt_bwd_dkdv": "alu",
+    "simt_bwd_prefix_increment": "alu",
+    "simt_bwd_suffix_increment": "alu",
 }
+METRIC_BWD = "KATA causal bwd (dq, dk, dv) tokens/sec at T=131072 (chunked)"
 
 
 def algorithmic_per_token_head(d_k, d_v, C, feature="psd"):
@@ -54,6 +59,22 @@ def algorithmic_per_token_head(d_k, d_v, C, feature="psd"):
     update = 2 * D * d_v + D
     readout = 2 * D * d_v + 2 * D
     return intra + update + readout, (2 * d_k + d_v) * 2 + d_v * 2
+
+
+def algorithmic_backward_per_token_head(d_k, d_v, C, feature="psd"):
+    """(flops, bytes) the gradient of the chunked forward must do per
+    token-head: the carried parts of dq (S g + z c, then the query feature's
+    Jacobian), dk (R v + r, the key feature's Jacobian) and dv (R^T phi(k)),
+    the updates of the prefix and suffix states, the normaliser and g, c; the
+    causal half of the intra-chunk pairs (q.k, g.v, dq, dk, dv, w); bf16 q, k,
+    v, dout read once and dq, dk, dv written once. The kernels also recompute
+    dout . y from the numerator; that recomputation is not counted."""
+    D = d_k * (d_k + 1) // 2 if feature == "psd" else d_k + 1
+    carried = (2 * D * d_v + 6 * D) + (2 * D * d_v + 6 * D) + (2 * D * d_v + D)
+    updates = (2 * D * d_v + 2 * D) + (2 * D * d_v + 3 * D)
+    norm = 2 * D + 3 * d_v
+    intra = (C + 1) / 2 * (6 * d_k + 4 * d_v + 4)
+    return carried + updates + norm + intra, (4 * d_k + 3 * d_v) * 2
 
 
 def load_peaks():
@@ -307,7 +328,17 @@ def run_ours(args, rank, world, local_rank):
     else:
         q, k, v = W.make_inputs(w, device=dev)
         o = torch.empty_like(v)
-        if form == "quadratic":
+        if form == "backward":
+            dy = W.make_grad_output(w, device=dev)            # seeded dL/dy
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            nb = api.bwd_chunked_workspace_bytes(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature)
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+            def step():
+                api.kata_bwd_chunked(q, k, v, dy, dq, dk, dv, w.C, w.feature, workspace=ws)
+            flops_th, bytes_th = algorithmic_backward_per_token_head(w.d_k, w.d_v, w.C, w.feature)
+            e2e_in, e2e_out = [q, k, v, dy], [dq, dk, dv]
+        elif form == "quadratic":
             ws = None
 
             def step():
@@ -327,7 +358,8 @@ def run_ours(args, rank, world, local_rank):
         config["form"] = {"chunked": "chunked (segmented scan carry)",
                           "sequential": "chunked (sequential carry)",
                           "first_order": "chunked first-order (segmented scan carry)",
-                          "quadratic": "quadratic (flash-style)"}[form]
+                          "quadratic": "quadratic (flash-style)",
+                          "backward": "gradient of the chunked form (prefix and suffix scans)"}[form]
 
     def barrier():
         if world > 1:
@@ -379,9 +411,14 @@ def run_ours(args, rank, world, local_rank):
         peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
         unit = "TFLOP/s"
         peak_kind = f"{peaks['source']} bf16 {'sustained' if sustained else 'burst'}"
+    scope = "dominant kernel (it carries the step's whole algorithmic work)"
+    if form == "backward":
+        # the work is split over four kernels: hold the whole step to the roofline
+        achieved = flops_th * per_launch_units / (ms / 1e3) / 1e12
+        scope = "whole step (four kernels share the work)"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": recorded_traffic(dom), "kernel": dom,
-                "kernel_ms": dom_ms / launches, "peak_kind": peak_kind,
+                "kernel_ms": dom_ms / launches, "peak_kind": peak_kind, "scope": scope,
                 "step_frac_of_tensor_or_hbm": None}
     # whole-step fraction of the binding tensor/HBM roofline of the method
     t_tensor = flops_th * token_heads / (peaks["bf16_tflops"] * 1e12)
@@ -392,17 +429,17 @@ def run_ours(args, rank, world, local_rank):
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e and form != "decode":
-        qh = q.cpu().pin_memory()
-        kh = k.cpu().pin_memory()
-        vh = v.cpu().pin_memory()
-        oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        if form != "backward":
+            e2e_in, e2e_out = [q, k, v], [o]
+        hosts_in = [t.cpu().pin_memory() for t in e2e_in]
+        hosts_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in e2e_out]
 
         def e2e_step():
-            q.copy_(qh, non_blocking=True)
-            k.copy_(kh, non_blocking=True)
-            v.copy_(vh, non_blocking=True)
+            for d, h in zip(e2e_in, hosts_in):
+                d.copy_(h, non_blocking=True)
             step()
-            oh.copy_(o, non_blocking=True)
+            for h, d in zip(hosts_out, e2e_out):
+                h.copy_(d, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -418,8 +455,9 @@ def run_ours(args, rank, world, local_rank):
         ms_e2e = s2.elapsed_time(e2) / n_e2e
         e2e_value, ms_e2e = aggregate_throughput(ms_e2e, tokens_per_step, world, dev)
         e2e = {"value": e2e_value, "unit": UNIT,
-               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (q, k, v)),
-               "d2h_bytes_per_step": o.numel() * o.element_size(), "ms_per_step": ms_e2e}
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in e2e_in),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in e2e_out),
+               "ms_per_step": ms_e2e}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and form == "chunked":
@@ -429,7 +467,7 @@ def run_ours(args, rank, world, local_rank):
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC_BWD if form == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config | {"parallelism": f"replicas x{world}"},
@@ -449,7 +487,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long131k_bf16")
     ap.add_argument("--form", default="chunked",
-                    choices=["chunked", "sequential", "first_order", "quadratic", "decode"],
+                    choices=["chunked", "sequential", "first_order", "quadratic", "decode", "backward"],
                     help="chunked is the headline; the others are secondary measurements")
     ap.add_argument("--decode-batch", type=int, default=W_DECODE_BATCH)
     ap.add_argument("--T", type=int, default=0, help="override T (profiling a smaller case)")

@@ -205,8 +205,54 @@ KATA_API kata_status_t kata_decode_step(const void *q, const void *k, const void
                                kata_stream_t stream);
 
 /*
- * Synchronises `stream`, then reads the status word a kata_fwd_chunked(...)
- * or kata_fwd_chunked_sequential(...) call left in `workspace`: KATA_OK, or
+ * Workspace bytes kata_bwd_chunked needs for this problem on the CURRENT
+ * device; 0 for an unsupported shape. Same alignment and exclusivity rules as
+ * the forward's workspace.
+ */
+KATA_API size_t kata_bwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C,
+                                                 kata_dtype_t dtype, kata_feature_t feature);
+
+/*
+ * Gradient of the causal forward: given dout = dL/dy for the output
+ * y of kata_fwd_chunked(q, k, v), writes dq = dL/dq, dk = dL/dk, dv = dL/dv.
+ * The pages pre-train language models on these kernels (arXiv abstract;
+ * explainer sections 3 and 4) without printing the backward; this is the
+ * chain rule of the definition above. With d_t = sum_{s<=t} w_ts,
+ *   g_t = dout_t / d_t,   c_t = -(dout_t . y_t) / d_t,
+ *   e_ts = g_t . v_s + c_t                        (dL/dw_ts, s <= t)
+ *   dv_s = sum_{t>=s} w_ts g_t
+ *   dq_t = sum_{s<=t} e_ts dw_ts/dq_t,   dk_s = sum_{t>=s} e_ts dw_ts/dk_s
+ * (dw/dq = 2 <q,k> k, dw/dk = 2 <q,k> q for PSD; k and q for FIRST_ORDER),
+ * evaluated in the exact chunked form: each sum is a dense block inside a
+ * chunk plus a state carried from the other chunks (the forward's prefix
+ * state for dq, a suffix state R = sum phi_q(q_t) g_t^T, r = sum phi_q(q_t)
+ * c_t carried backwards for dk and dv), both through the segment scan. The
+ * forward's output is not an input: d_t and dout_t . y_t are recomputed in
+ * fp32 (a stored bf16 y would enter c_t with its rounding, which the
+ * cancellation in e_ts amplifies by 1 / d_t).
+ *
+ *   q, k, v            device, the forward's inputs (layouts above).
+ *   dout               device [B, H, T, d_v], dtype.
+ *   dq, dk / dv        device [B, H, T, d_k] / [B, H, T, d_v], dtype,
+ *                      written (may not alias the inputs).
+ *   workspace          device, >= kata_bwd_chunked_workspace_bytes(...),
+ *                      256-byte aligned, contents on entry ignored; holds the
+ *                      status word afterwards (kata_workspace_status reports
+ *                      a non-positive normaliser as for the forward).
+ * Arithmetic is fp32 (CUDA cores) for both dtypes. Returns KATA_OK when the
+ * work was launched; B, H or T = 0 launches nothing.
+ */
+KATA_API kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
+                                        const void *dout, void *dq, void *dk, void *dv,
+                                        int B, int H, int T, int d_k, int d_v, int C,
+                                        kata_dtype_t dtype, kata_feature_t feature,
+                                        void *workspace, size_t workspace_bytes,
+                                        kata_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the status word a kata_fwd_chunked(...),
+ * kata_fwd_chunked_sequential(...) or kata_bwd_chunked(...) call left in
+ * `workspace`: KATA_OK, or
  * KATA_ERR_NONPOSITIVE_NORMALISER if any row had a normaliser <= 0, or
  * KATA_ERR_CUDA if the synchronisation or the copy failed.
  */

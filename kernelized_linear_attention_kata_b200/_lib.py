@@ -41,6 +41,9 @@ SIGNATURES = {
                                                 _fp, _fp, _vp]),
     "kata_fwd_quadratic": (ctypes.c_int, [_cvp, _cvp, _cvp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "kata_decode_step": (ctypes.c_int, [_cvp, _cvp, _cvp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+    "kata_bwd_chunked_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "kata_bwd_chunked": (ctypes.c_int, [_cvp, _cvp, _cvp, _cvp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                        _i, _i, _i, _i, _vp, _sz, _vp]),
     "kata_workspace_status": (ctypes.c_int, [_cvp, _vp]),
     "kata_profile_enable": (ctypes.c_int, [_i]),
     "kata_profile_count": (ctypes.c_int, []),

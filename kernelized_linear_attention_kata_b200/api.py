@@ -129,6 +129,32 @@ def kata_decode_step(q, k, v, S, z, y, feature="psd", stream=None):
     return y
 
 
+def bwd_chunked_workspace_bytes(B, H, T, d_k, d_v, C, dtype=torch.bfloat16, feature="psd") -> int:
+    return int(lib().kata_bwd_chunked_workspace_bytes(B, H, T, d_k, d_v, C, _DTYPES[dtype],
+                                                      _feature(feature)))
+
+
+def kata_bwd_chunked(q, k, v, dout, dq, dk, dv, C, feature="psd", workspace=None, stream=None):
+    """Gradient of the chunked forward into dq, dk, dv (see include/kata.h)."""
+    B, H, T, d_k, d_v = _shapes(q, k, v, dout)
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
+        raise ValueError("dq, dk, dv must have the shapes of q, k, v")
+    for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must be {q.dtype}")
+    if workspace is None:
+        n = bwd_chunked_workspace_bytes(B, H, T, d_k, d_v, C, q.dtype, feature)
+        if n == 0:
+            raise ValueError("unsupported shape for kata_bwd_chunked")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    st = lib().kata_bwd_chunked(
+        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(dout, "dout"), _dev(dq, "dq"),
+        _dev(dk, "dk"), _dev(dv, "dv"), B, H, T, d_k, d_v, C, _dtype(q), _feature(feature),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream))
+    check("kata_bwd_chunked", st)
+    return dq, dk, dv
+
+
 def kata_workspace_status(workspace, stream=None) -> int:
     """Synchronises the stream and returns the status code left in the workspace."""
     return int(lib().kata_workspace_status(_dev(workspace, "workspace"), _stream(stream)))
@@ -173,6 +199,12 @@ def fwd_quadratic(q, k, v, feature="psd"):
     return kata_fwd_quadratic(q, k, v, o, feature)
 
 
+def bwd_chunked(q, k, v, dout, C, feature="psd"):
+    """(dq, dk, dv) of sum(dout * y) for y = fwd_chunked(q, k, v)."""
+    return kata_bwd_chunked(q, k, v, dout, torch.empty_like(q), torch.empty_like(k),
+                            torch.empty_like(v), C, feature)
+
+
 def decode_step(q, k, v, S, z, feature="psd"):
     y = torch.empty_like(v)
     return kata_decode_step(q, k, v, S, z, y, feature)
@@ -182,4 +214,5 @@ __all__ = [
     "state_dim", "chunked_workspace_bytes", "alloc_workspace", "kata_fwd_chunked",
     "kata_fwd_chunked_sequential", "kata_fwd_quadratic", "kata_decode_step",
     "kata_workspace_status", "profile_enable", "profile_read", "fwd_chunked", "fwd_quadratic", "decode_step", "_lib",
+    "bwd_chunked_workspace_bytes", "kata_bwd_chunked", "bwd_chunked",
 ]

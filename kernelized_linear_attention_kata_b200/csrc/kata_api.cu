@@ -69,6 +69,23 @@ size_t workspace_bytes_for(long long BH, int D, int d_k, int d_v, const Split &s
   return kHeaderBytes + align_up(agg, kAlign);
 }
 
+// Backward workspace: status header | prefix-state increments | suffix-state
+// increments (each [BH][G][D][d_v + 1] fp32) | normalisers d_t [BH][T] fp32 |
+// c_t [BH][T] fp32.
+struct BwdLayout {
+  size_t agg_bytes, den_bytes;
+  size_t aggS() const { return kHeaderBytes; }
+  size_t aggR() const { return kHeaderBytes + agg_bytes; }
+  size_t den() const { return kHeaderBytes + 2 * agg_bytes; }
+  size_t c() const { return kHeaderBytes + 2 * agg_bytes + den_bytes; }
+  size_t total() const { return kHeaderBytes + 2 * agg_bytes + 2 * den_bytes; }
+};
+
+BwdLayout bwd_layout(long long BH, int T, int D, int d_v, const Split &sp) {
+  return {align_up((size_t)BH * (size_t)sp.G * (size_t)D * (size_t)(d_v + 1) * sizeof(float), kAlign),
+          align_up((size_t)BH * (size_t)T * sizeof(float), kAlign)};
+}
+
 // Calls F::template run<DK, DV, FEAT>() for the runtime (d_k, d_v, feature).
 template <typename F>
 kata_status_t dispatch_shape(int d_k, int d_v, kata_feature_t feature, F &&f) {
@@ -114,6 +131,16 @@ struct QuadraticRun {
     if (e == cudaErrorNotSupported)
       e = dtype == KATA_DTYPE_F32 ? simt_quadratic<DK, DV, FEAT, float>(a)
                                   : simt_quadratic<DK, DV, FEAT, __nv_bfloat16>(a);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+  }
+};
+
+struct BackwardRun {
+  kata_dtype_t dtype;
+  BackwardLaunch a;
+  template <int DK, int DV, int FEAT> kata_status_t operator()() {
+    const cudaError_t e = dtype == KATA_DTYPE_F32 ? simt_backward<DK, DV, FEAT, float>(a)
+                                                  : simt_backward<DK, DV, FEAT, __nv_bfloat16>(a);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
   }
 };
@@ -243,6 +270,48 @@ kata_status_t kata_decode_step(const void *q, const void *k, const void *v, floa
   if (reinterpret_cast<uintptr_t>(S) % 16 != 0) return KATA_ERR_INVALID_ARGUMENT;
   if (BH > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
   DecodeRun run{dtype, DecodeLaunch{q, k, v, S, z, y, BH, stream}};
+  return dispatch_shape(d_k, d_v, feature, run);
+}
+
+size_t kata_bwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C,
+                                        kata_dtype_t dtype, kata_feature_t feature) {
+  if (B < 0 || H < 0 || T < 0 || C <= 0) return 0;
+  if (!supported(d_k, d_v, C, dtype, feature)) return 0;
+  const int sms = device_sm_count();
+  if (sms <= 0) return 0;
+  const long long BH = (long long)B * H;
+  const Split sp = segment_split(BH, T, C, sms, false);
+  return bwd_layout(BH, T, (int)kata_state_dim(d_k, feature), d_v, sp).total();
+}
+
+kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
+                               const void *dout, void *dq, void *dk, void *dv, int B, int H,
+                               int T, int d_k, int d_v, int C, kata_dtype_t dtype,
+                               kata_feature_t feature, void *workspace, size_t workspace_bytes,
+                               kata_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || H < 0 || T < 0 || C <= 0) return KATA_ERR_INVALID_ARGUMENT;
+  if (!supported(d_k, d_v, C, dtype, feature)) return KATA_ERR_UNSUPPORTED;
+  if (!workspace) return KATA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return KATA_ERR_WORKSPACE;
+  const int sms = device_sm_count();
+  if (sms <= 0) return KATA_ERR_CUDA;
+  const long long BH = (long long)B * H;
+  const Split sp = segment_split(BH, T, C, sms, false);
+  const BwdLayout lay = bwd_layout(BH, T, (int)kata_state_dim(d_k, feature), d_v, sp);
+  if (workspace_bytes < lay.total()) return KATA_ERR_WORKSPACE;
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  if (cudaMemsetAsync(ws, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
+  if (BH == 0 || T == 0) return KATA_OK;
+  if (!q || !k || !v || !dout || !dq || !dk || !dv) return KATA_ERR_INVALID_ARGUMENT;
+  if (BH * (long long)sp.G > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
+  BackwardRun run{dtype, BackwardLaunch{q, k, v, dout, dq, dk, dv, BH, T,
+                                        reinterpret_cast<unsigned *>(ws),
+                                        reinterpret_cast<float *>(ws + lay.aggS()),
+                                        reinterpret_cast<float *>(ws + lay.aggR()),
+                                        reinterpret_cast<float *>(ws + lay.den()),
+                                        reinterpret_cast<float *>(ws + lay.c()), sp.G, sp.seg_len,
+                                        stream}};
   return dispatch_shape(d_k, d_v, feature, run);
 }
 

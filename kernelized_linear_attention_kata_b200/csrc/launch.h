@@ -36,6 +36,21 @@ struct DecodeLaunch {
   cudaStream_t stream;
 };
 
+// Gradient of the chunked forward: q, k, v, dout in; dq, dk, dv out (all in
+// the element type). Workspace regions: segment increments of the prefix
+// state (aggS) and of the suffix state (aggR), each [BH][G][D][d_v + 1], and
+// per token the normaliser d_t and c_t = -(dout_t . y_t) / d_t, [BH][T] each.
+struct BackwardLaunch {
+  const void *q, *k, *v, *dout;
+  void *dq, *dk, *dv;
+  long long BH;
+  int T;
+  unsigned *status;
+  float *aggS, *aggR, *den, *c;
+  int G, seg_len;
+  cudaStream_t stream;
+};
+
 // Tensor-core kernels (bf16 only). They return cudaErrorNotSupported, having
 // launched nothing, for shapes or alignments they do not handle; the caller
 // then runs the CUDA-core kernel instead.
@@ -50,5 +65,6 @@ size_t fo_tc_agg_floats();        // floats of one segment increment
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_chunked(const ChunkedLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_quadratic(const QuadraticLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_decode(const DecodeLaunch &a);
+template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_backward(const BackwardLaunch &a);
 
 }  // namespace kata

@@ -126,6 +126,13 @@ def make_inputs(w: Workload, device="cpu"):
     return (q.to(dt).contiguous(), k.to(dt).contiguous(), v.to(dt).contiguous())
 
 
+def make_grad_output(w: Workload, device="cpu"):
+    """Upstream gradient dL/dy for the backward, [B, H, T, d_v] N(0,1) in the
+    workload dtype, seeded apart from the inputs."""
+    g = _generator(w.seed + 7919, device)
+    return _randn((w.B, w.H, w.T, w.d_v), g, device).to(w.torch_dtype).contiguous()
+
+
 def make_decode_inputs(batch=DECODE_BATCH, heads=DECODE_HEADS, d_k=DECODE_DK, d_v=DECODE_DV,
                        seed=DECODE_SEED, device="cpu", dtype=torch.bfloat16):
     """The decode step's token: q, k unit [batch, H, d_k]; v N(0,1) [batch, H, d_v]."""

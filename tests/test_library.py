@@ -33,7 +33,8 @@ def test_header_declares_the_abi():
     names = declared_symbols()
     for required in ("kata_fwd_chunked", "kata_fwd_quadratic", "kata_decode_step",
                      "kata_state_dim", "kata_fwd_chunked_workspace_bytes",
-                     "kata_workspace_status", "kata_status_string"):
+                     "kata_workspace_status", "kata_status_string", "kata_bwd_chunked",
+                     "kata_bwd_chunked_workspace_bytes"):
         assert required in names
 
 
@@ -94,6 +95,28 @@ def test_host_rejects_bad_arguments(lib):
     assert lib.kata_fwd_quadratic(p, p, p, p, -1, 1, 8, 32, 64, 1, 0, None) == L.KATA_ERR_INVALID_ARGUMENT
     assert lib.kata_decode_step(p, p, p, p, p, p, 1, -2, 32, 64, 1, 0, None) == L.KATA_ERR_INVALID_ARGUMENT
     assert lib.kata_workspace_status(None, None) == L.KATA_ERR_WORKSPACE
+
+
+def _bwd(lib, d_k=32, d_v=64, C=64, dtype=L.KATA_DTYPE_BF16, feature=L.KATA_FEATURE_PSD, B=1, H=1,
+         T=16, ws=None):
+    p = ctypes.c_void_p(256)
+    return lib.kata_bwd_chunked(p, p, p, p, p, p, p, B, H, T, d_k, d_v, C, dtype, feature,
+                                ws if ws is not None else p, 1 << 20, None)
+
+
+def test_backward_host_checks(lib):
+    assert _bwd(lib, d_k=24) == L.KATA_ERR_UNSUPPORTED
+    assert _bwd(lib, d_k=64) == L.KATA_ERR_UNSUPPORTED           # PSD d_k = 64 not built
+    assert _bwd(lib, d_v=48) == L.KATA_ERR_UNSUPPORTED
+    assert _bwd(lib, feature=3) == L.KATA_ERR_UNSUPPORTED
+    assert _bwd(lib, dtype=5) == L.KATA_ERR_UNSUPPORTED
+    assert _bwd(lib, B=-1) == L.KATA_ERR_INVALID_ARGUMENT
+    assert _bwd(lib, T=-3) == L.KATA_ERR_INVALID_ARGUMENT
+    assert _bwd(lib, C=0) == L.KATA_ERR_INVALID_ARGUMENT
+    assert _bwd(lib, ws=ctypes.c_void_p(0)) == L.KATA_ERR_WORKSPACE
+    assert _bwd(lib, ws=ctypes.c_void_p(256 + 8)) == L.KATA_ERR_WORKSPACE
+    assert lib.kata_bwd_chunked_workspace_bytes(1, 1, 16, 24, 64, 64, 1, 0) == 0
+    assert lib.kata_bwd_chunked_workspace_bytes(-1, 1, 16, 32, 64, 64, 1, 0) == 0
 
 
 def test_empty_problems_launch_nothing(lib):
