@@ -147,6 +147,40 @@ KATA_API kata_status_t kata_fwd_chunked_sequential(const void *q, const void *k,
                                           kata_stream_t stream);
 
 /*
+ * The same forward starting from a given state instead of zero: the carry
+ * into every chunk is S0 + (the increments of the earlier chunks), i.e. the
+ * sequence continues one whose state after its last token is (S0, z0). This
+ * is how a sequence cut into slices (one per GPU) is processed: slice r
+ * starts from the sum of the states of slices 0 .. r-1 (the scan across
+ * chunks, explainer 2.3, taken one level up).
+ *   S0, z0             device fp32 [B, H, D, d_v] and [B, H, D], library
+ *                      layout (read only); either may be NULL (zero).
+ * Everything else as kata_fwd_chunked; S_out / z_out include S0 / z0, and
+ * with T = 0 they are copies of S0 / z0.
+ */
+KATA_API kata_status_t kata_fwd_chunked_from_state(const void *q, const void *k, const void *v,
+                                                   void *o, int B, int H, int T, int d_k, int d_v,
+                                                   int C, kata_dtype_t dtype, kata_feature_t feature,
+                                                   const float *S0, const float *z0,
+                                                   float *S_out, float *z_out,
+                                                   void *workspace, size_t workspace_bytes,
+                                                   kata_stream_t stream);
+
+/*
+ * Only the state after the T tokens: S_out = sum_t phi(k_t) v_t^T and
+ * z_out = sum_t phi(k_t) (library layout), without computing outputs. The
+ * state is a sum over tokens, so it is computed as per-segment increments
+ * reduced per head; a sequence slice's state is what the slices after it
+ * need as their starting state. q and o are not inputs. Same workspace as
+ * kata_fwd_chunked (kata_fwd_chunked_workspace_bytes is enough).
+ */
+KATA_API kata_status_t kata_chunked_state(const void *k, const void *v, int B, int H, int T,
+                                          int d_k, int d_v, int C, kata_dtype_t dtype,
+                                          kata_feature_t feature, float *S_out, float *z_out,
+                                          void *workspace, size_t workspace_bytes,
+                                          kata_stream_t stream);
+
+/*
  * kata_fwd_chunked without a caller-provided workspace, for callers that
  * cannot allocate device memory (for example a host application whose device
  * memory belongs entirely to another runtime's pool, or latency-critical code

@@ -39,6 +39,10 @@ SIGNATURES = {
     "kata_fwd_chunked_sequential": (ctypes.c_int, _FWD),
     "kata_fwd_chunked_noalloc": (ctypes.c_int, [_cvp, _cvp, _cvp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                                                 _fp, _fp, _vp]),
+    "kata_fwd_chunked_from_state": (ctypes.c_int, [_cvp, _cvp, _cvp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                                   _i, _fp, _fp, _fp, _fp, _vp, _sz, _vp]),
+    "kata_chunked_state": (ctypes.c_int, [_cvp, _cvp, _i, _i, _i, _i, _i, _i, _i, _i, _fp, _fp, _vp,
+                                          _sz, _vp]),
     "kata_fwd_quadratic": (ctypes.c_int, [_cvp, _cvp, _cvp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "kata_decode_step": (ctypes.c_int, [_cvp, _cvp, _cvp, _fp, _fp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "kata_bwd_chunked_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i, _i]),

@@ -84,19 +84,56 @@ def _shapes(q, k, v, o):
     return B, H, T, d_k, v.shape[3]
 
 
+def _state_shapes(B, H, d_k, d_v, feature, S, z, names):
+    D = state_dim(d_k, feature)
+    if S is not None and tuple(S.shape) != (B, H, D, d_v):
+        raise ValueError(f"{names[0]} must be [B,H,{D},{d_v}] fp32")
+    if z is not None and tuple(z.shape) != (B, H, D):
+        raise ValueError(f"{names[1]} must be [B,H,{D}] fp32")
+
+
 def kata_fwd_chunked(q, k, v, o, C, feature="psd", S_out=None, z_out=None, workspace=None,
-                     stream=None, sequential=False):
-    """Chunked-state causal forward into `o` (see include/kata.h)."""
+                     stream=None, sequential=False, S0=None, z0=None):
+    """Chunked-state causal forward into `o` (see include/kata.h); with S0 / z0
+    it starts from that state (kata_fwd_chunked_from_state)."""
     B, H, T, d_k, d_v = _shapes(q, k, v, o)
+    _state_shapes(B, H, d_k, d_v, feature, S_out, z_out, ("S_out", "z_out"))
     if workspace is None:
         workspace = alloc_workspace(B, H, T, d_k, d_v, C, q.dtype, feature, q.device)
-    fn = "kata_fwd_chunked_sequential" if sequential else "kata_fwd_chunked"
-    st = getattr(lib(), fn)(
-        _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d_k, d_v, C, _dtype(q),
-        _feature(feature), _opt(S_out, "S_out"), _opt(z_out, "z_out"), _dev(workspace, "workspace"),
-        workspace.numel() * workspace.element_size(), _stream(stream))
+    ws = (_dev(workspace, "workspace"), workspace.numel() * workspace.element_size())
+    if S0 is not None or z0 is not None:
+        if sequential:
+            raise ValueError("the sequential-carry entry point takes no initial state")
+        _state_shapes(B, H, d_k, d_v, feature, S0, z0, ("S0", "z0"))
+        fn = "kata_fwd_chunked_from_state"
+        st = lib().kata_fwd_chunked_from_state(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d_k, d_v, C, _dtype(q),
+            _feature(feature), _opt(S0, "S0"), _opt(z0, "z0"), _opt(S_out, "S_out"),
+            _opt(z_out, "z_out"), *ws, _stream(stream))
+    else:
+        fn = "kata_fwd_chunked_sequential" if sequential else "kata_fwd_chunked"
+        st = getattr(lib(), fn)(
+            _dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), B, H, T, d_k, d_v, C, _dtype(q),
+            _feature(feature), _opt(S_out, "S_out"), _opt(z_out, "z_out"), *ws, _stream(stream))
     check(fn, st)
     return o
+
+
+def kata_chunked_state(k, v, S_out, z_out, C, feature="psd", workspace=None, stream=None):
+    """State after all tokens of k, v (no outputs) into S_out, z_out."""
+    if k.dim() != 4 or v.dim() != 4 or v.shape[:3] != k.shape[:3] or k.dtype != v.dtype:
+        raise ValueError("expected k [B,H,T,d_k] and v [B,H,T,d_v] of one dtype")
+    B, H, T, d_k = k.shape
+    d_v = v.shape[3]
+    _state_shapes(B, H, d_k, d_v, feature, S_out, z_out, ("S_out", "z_out"))
+    if workspace is None:
+        workspace = alloc_workspace(B, H, T, d_k, d_v, C, k.dtype, feature, k.device)
+    st = lib().kata_chunked_state(
+        _dev(k, "k"), _dev(v, "v"), B, H, T, d_k, d_v, C, _dtype(k), _feature(feature),
+        _opt(S_out, "S_out"), _opt(z_out, "z_out"), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    check("kata_chunked_state", st)
+    return S_out, z_out
 
 
 def kata_fwd_chunked_sequential(q, k, v, o, C, feature="psd", S_out=None, z_out=None,
@@ -194,6 +231,15 @@ def fwd_chunked(q, k, v, C, feature="psd", return_state=False, sequential=False)
     return o
 
 
+def chunked_state(k, v, C, feature="psd"):
+    """(S, z): the state after all tokens, allocated with torch."""
+    B, H, _, d_k = k.shape
+    D = state_dim(d_k, feature)
+    S = torch.empty((B, H, D, v.shape[3]), dtype=torch.float32, device=k.device)
+    z = torch.empty((B, H, D), dtype=torch.float32, device=k.device)
+    return kata_chunked_state(k, v, S, z, C, feature)
+
+
 def fwd_quadratic(q, k, v, feature="psd"):
     o = torch.empty_like(v)
     return kata_fwd_quadratic(q, k, v, o, feature)
@@ -214,5 +260,6 @@ __all__ = [
     "state_dim", "chunked_workspace_bytes", "alloc_workspace", "kata_fwd_chunked",
     "kata_fwd_chunked_sequential", "kata_fwd_quadratic", "kata_decode_step",
     "kata_workspace_status", "profile_enable", "profile_read", "fwd_chunked", "fwd_quadratic", "decode_step", "_lib",
-    "bwd_chunked_workspace_bytes", "kata_bwd_chunked", "bwd_chunked",
+    "bwd_chunked_workspace_bytes", "kata_bwd_chunked", "bwd_chunked", "kata_chunked_state",
+    "chunked_state",
 ]

@@ -259,7 +259,8 @@ template <bool AGG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-                  float *__restrict__ agg, float *__restrict__ S_out, float *__restrict__ z_out,
+                  float *__restrict__ agg, const float *__restrict__ S0, const float *__restrict__ z0,
+                  float *__restrict__ S_out, float *__restrict__ z_out,
                   unsigned *__restrict__ status, int T, int G_grid, int G_total, int seg_len) {
   using L = Layout<AGG>;
   constexpr int NK = L::kKRingSlots;
@@ -683,7 +684,9 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     uint8_t *zsnap = smem + L::kOffZSnap;
     bool ok = true;
 
-    // ---- carry-in: sum of the increments of segments 0 .. g-1 ----
+    // ---- carry-in: the initial state (library layout, if any; features
+    //      doubled off the diagonal as inside the kernel) plus the increments
+    //      of segments 0 .. g-1 ----
     {
       const float *seg0 = agg + (size_t)bh * G_total * kAggFloats;
 #pragma unroll 1
@@ -694,6 +697,12 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
           float acc[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+          if (!AGG && f < kD && S0) {
+            const float *s0 = S0 + ((size_t)bh * kD + abi_row(f)) * kDV + 16 * q4;
+            const float mf = f < kDK ? 1.f : 2.f;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) acc[c] = mf * s0[c];
+          }
           if (!AGG && f < kD) {
             for (int gp = 0; gp < g; ++gp) {
               const float4 *src =
@@ -723,6 +732,14 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         float acc[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+        if (!AGG && r < kDK && z0) {
+          // Z_rc = z_(min, max) (the library's packed row of the pair)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int i = r < c ? r : c, j = r < c ? c : r;
+            acc[c] = z0[(size_t)bh * kD + i * kDK - i * (i - 1) / 2 + (j - i)];
+          }
+        }
         if (!AGG && r < kDK) {
           for (int gp = 0; gp < g; ++gp) {
             const float4 *src =
@@ -902,31 +919,38 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
   const int per = (nchunks + G - 1) / G;
   G = (nchunks + per - 1) / per;
   const int seg_len = per * kC;
+  // the state-only call reads neither q nor o: their maps are built on k, v
+  // and never used by the increment kernel
   CUtensorMap tq, tk, tv, to;
-  if (!make_tma_3d_bf16(&tq, a.q, kDK, a.T, a.BH, kC) ||
+  if (!make_tma_3d_bf16(&tq, a.state_only ? a.k : a.q, kDK, a.T, a.BH, kC) ||
       !make_tma_3d_bf16(&tk, a.k, kDK, a.T, a.BH, kC) ||
       !make_tma_3d_bf16(&tv, a.v, kDV, a.T, a.BH, kC) ||
-      !make_tma_3d_bf16(&to, a.o, kDV, a.T, a.BH, kC))
+      !make_tma_3d_bf16(&to, a.state_only ? a.v : a.o, kDV, a.T, a.BH, kC))
     return cudaErrorNotSupported;
   cudaError_t e;
-  if (G > 1) {
+  // increments of segments 0 .. G-2 (all G for the state-only call)
+  const int G_inc = a.state_only ? G : G - 1;
+  if (G_inc > 0) {
     auto kagg = chunked_tc_kernel<true>;
     e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Layout<true>::kSmemBytes);
     if (e != cudaSuccess) return e;
     ProfileScope prof("tc_segment_increment", a.stream);
-    kagg<<<(unsigned)(a.BH * (G - 1)), kThreads, Layout<true>::kSmemBytes, a.stream>>>(
-        tq, tk, tv, to, a.agg, nullptr, nullptr, a.status, a.T, G - 1, G, seg_len);
+    kagg<<<(unsigned)(a.BH * G_inc), kThreads, Layout<true>::kSmemBytes, a.stream>>>(
+        tq, tk, tv, to, a.agg, nullptr, nullptr, nullptr, nullptr, a.status, a.T, G_inc, G,
+        seg_len);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  if (a.state_only)
+    return state_reduce(kAggPsdTc, a.agg, a.BH, G, kD, kDK, kDV, a.S_out, a.z_out, 0.f, a.stream);
   auto kpass = chunked_tc_kernel<false>;
   e = cudaFuncSetAttribute(kpass, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Layout<false>::kSmemBytes);
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_segment_pass", a.stream);
   kpass<<<(unsigned)(a.BH * G), kThreads, Layout<false>::kSmemBytes, a.stream>>>(
-      tq, tk, tv, to, a.agg, a.S_out, a.z_out, a.status, a.T, G, G, seg_len);
+      tq, tk, tv, to, a.agg, a.S0, a.z0, a.S_out, a.z_out, a.status, a.T, G, G, seg_len);
   return cudaGetLastError();
 }
 

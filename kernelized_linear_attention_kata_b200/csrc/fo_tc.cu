@@ -113,7 +113,8 @@ template <bool AGG>
 __global__ void __launch_bounds__(kThreads, 1)
 fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
              const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-             float *__restrict__ agg, float *__restrict__ S_out, float *__restrict__ z_out,
+             float *__restrict__ agg, const float *__restrict__ S0, const float *__restrict__ z0,
+             float *__restrict__ S_out, float *__restrict__ z_out,
              unsigned *__restrict__ status, int T, int G_grid, int G_total, int seg_len) {
   using L = FoLayout<AGG>;
   extern __shared__ uint8_t smem_raw[];
@@ -363,12 +364,23 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       }
     };
 
-    // ---- carry-in: S' = sum of the increments of segments 0 .. g-1 ----
+    // ---- carry-in: S' = the initial state (library layout, if any) plus the
+    //      increments of segments 0 .. g-1 ----
     if (!AGG) {
       const float *seg0 = agg + (size_t)bh * G_total * kAggFloats;
       float acc[kNa];
 #pragma unroll
       for (int c = 0; c < kNa; ++c) acc[c] = 0.f;
+      if (r < kRows) {
+        // library row 0 is the constant feature (internal row 64), row 1 + f is k_f
+        const int lr = r == kDh ? 0 : r + 1;
+        if (S0) {
+          const float *s0 = S0 + ((size_t)bh * kRows + lr) * kDh;
+#pragma unroll
+          for (int c = 0; c < kDh; ++c) acc[c] = s0[c];
+        }
+        if (z0) acc[kDh] = z0[(size_t)bh * kRows + lr];
+      }
       if (r < kRows)
         for (int gp = 0; gp < g; ++gp) {
           const float *src = seg0 + (size_t)gp * kAggFloats + (size_t)r * kRows;
@@ -510,29 +522,40 @@ cudaError_t fo_tc(const ChunkedLaunch &a) {
   const int per = (ntiles + G - 1) / G;
   G = (ntiles + per - 1) / per;
   const int seg_len = per * kTile;
+  // the state-only call reads neither q nor o: their maps are built on k, v
+  // and never used by the increment kernel
   CUtensorMap tq, tk, tv, to;
-  if (!make_tma_3d_bf16(&tq, a.q, kDh, a.T, a.BH, kTile) ||
+  if (!make_tma_3d_bf16(&tq, a.state_only ? a.k : a.q, kDh, a.T, a.BH, kTile) ||
       !make_tma_3d_bf16(&tk, a.k, kDh, a.T, a.BH, kTile) ||
       !make_tma_3d_bf16(&tv, a.v, kDh, a.T, a.BH, kTile) ||
-      !make_tma_3d_bf16(&to, a.o, kDh, a.T, a.BH, kTile))
+      !make_tma_3d_bf16(&to, a.state_only ? a.v : a.o, kDh, a.T, a.BH, kTile))
     return cudaErrorNotSupported;
   cudaError_t e;
-  if (G > 1) {
+  // increments of segments 0 .. G-2 (all G for the state-only call)
+  const int G_inc = a.state_only ? G : G - 1;
+  if (G_inc > 0) {
     auto kagg = fo_tc_kernel<true>;
     e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize, FoLayout<true>::kSmemBytes);
     if (e != cudaSuccess) return e;
     ProfileScope prof("tc_fo_increment", a.stream);
-    kagg<<<(unsigned)(a.BH * (G - 1)), kThreads, FoLayout<true>::kSmemBytes, a.stream>>>(
-        tq, tk, tv, to, a.agg, nullptr, nullptr, a.status, a.T, G - 1, G, seg_len);
+    kagg<<<(unsigned)(a.BH * G_inc), kThreads, FoLayout<true>::kSmemBytes, a.stream>>>(
+        tq, tk, tv, to, a.agg, nullptr, nullptr, nullptr, nullptr, a.status, a.T, G_inc, G, seg_len);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+  }
+  if (a.state_only) {
+    // the constant feature of the last segment's padded rows entered the count
+    const int t0_last = (G - 1) * seg_len;
+    const int last_tiles = (a.T - t0_last + kTile - 1) / kTile;
+    const float pad = (float)(last_tiles * kTile - (a.T - t0_last));
+    return state_reduce(kAggFoTc, a.agg, a.BH, G, kRows, kDh, kDh, a.S_out, a.z_out, pad, a.stream);
   }
   auto kpass = fo_tc_kernel<false>;
   e = cudaFuncSetAttribute(kpass, cudaFuncAttributeMaxDynamicSharedMemorySize, FoLayout<false>::kSmemBytes);
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_fo_pass", a.stream);
   kpass<<<(unsigned)(a.BH * G), kThreads, FoLayout<false>::kSmemBytes, a.stream>>>(
-      tq, tk, tv, to, a.agg, a.S_out, a.z_out, a.status, a.T, G, G, seg_len);
+      tq, tk, tv, to, a.agg, a.S0, a.z0, a.S_out, a.z_out, a.status, a.T, G, G, seg_len);
   return cudaGetLastError();
 }
 

@@ -158,7 +158,9 @@ struct DecodeRun {
 kata_status_t chunked_common(const void *q, const void *k, const void *v, void *o, int B, int H,
                              int T, int d_k, int d_v, int C, kata_dtype_t dtype,
                              kata_feature_t feature, float *S_out, float *z_out, void *workspace,
-                             size_t workspace_bytes, kata_stream_t stream_, bool sequential) {
+                             size_t workspace_bytes, kata_stream_t stream_, bool sequential,
+                             const float *S0 = nullptr, const float *z0 = nullptr,
+                             bool state_only = false) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (B < 0 || H < 0 || T < 0 || C <= 0) return KATA_ERR_INVALID_ARGUMENT;
   if (!supported(d_k, d_v, C, dtype, feature)) return KATA_ERR_UNSUPPORTED;
@@ -172,21 +174,28 @@ kata_status_t chunked_common(const void *q, const void *k, const void *v, void *
   if (workspace_bytes < workspace_bytes_for(BH, D, d_k, d_v, sp)) return KATA_ERR_WORKSPACE;
   unsigned char *ws = static_cast<unsigned char *>(workspace);
   if (BH == 0 || T == 0) {
+    // no tokens: the state out is the initial state (zero if none is given)
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
+    const size_t sb = (size_t)BH * D * d_v * sizeof(float), zb = (size_t)BH * D * sizeof(float);
     if (S_out && BH > 0 &&
-        cudaMemsetAsync(S_out, 0, (size_t)BH * D * d_v * sizeof(float), stream) != cudaSuccess)
+        (S0 ? cudaMemcpyAsync(S_out, S0, sb, cudaMemcpyDeviceToDevice, stream)
+            : cudaMemsetAsync(S_out, 0, sb, stream)) != cudaSuccess)
       return KATA_ERR_CUDA;
     if (z_out && BH > 0 &&
-        cudaMemsetAsync(z_out, 0, (size_t)BH * D * sizeof(float), stream) != cudaSuccess)
+        (z0 ? cudaMemcpyAsync(z_out, z0, zb, cudaMemcpyDeviceToDevice, stream)
+            : cudaMemsetAsync(z_out, 0, zb, stream)) != cudaSuccess)
       return KATA_ERR_CUDA;
     return KATA_OK;
   }
-  if (!q || !k || !v || !o) return KATA_ERR_INVALID_ARGUMENT;
+  if (!k || !v || (!state_only && (!q || !o))) return KATA_ERR_INVALID_ARGUMENT;
   unsigned *status = reinterpret_cast<unsigned *>(ws);
   if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
-  ChunkedRun run{dtype, ChunkedLaunch{q, k, v, o, BH, T, C, S_out, z_out, status,
-                                      reinterpret_cast<float *>(ws + kHeaderBytes), sp.G,
-                                      sp.seg_len, stream}};
+  ChunkedLaunch a{q, k, v, o, BH, T, C, S_out, z_out, status,
+                  reinterpret_cast<float *>(ws + kHeaderBytes), sp.G, sp.seg_len, stream};
+  a.S0 = S0;
+  a.z0 = z0;
+  a.state_only = state_only;
+  ChunkedRun run{dtype, a};
   return dispatch_shape(d_k, d_v, feature, run);
 }
 
@@ -242,6 +251,24 @@ kata_status_t kata_fwd_chunked_sequential(const void *q, const void *k, const vo
                                           size_t workspace_bytes, kata_stream_t stream) {
   return chunked_common(q, k, v, o, B, H, T, d_k, d_v, C, dtype, feature, S_out, z_out, workspace,
                         workspace_bytes, stream, true);
+}
+
+kata_status_t kata_fwd_chunked_from_state(const void *q, const void *k, const void *v, void *o,
+                                          int B, int H, int T, int d_k, int d_v, int C,
+                                          kata_dtype_t dtype, kata_feature_t feature,
+                                          const float *S0, const float *z0, float *S_out,
+                                          float *z_out, void *workspace, size_t workspace_bytes,
+                                          kata_stream_t stream) {
+  return chunked_common(q, k, v, o, B, H, T, d_k, d_v, C, dtype, feature, S_out, z_out, workspace,
+                        workspace_bytes, stream, false, S0, z0);
+}
+
+kata_status_t kata_chunked_state(const void *k, const void *v, int B, int H, int T, int d_k,
+                                 int d_v, int C, kata_dtype_t dtype, kata_feature_t feature,
+                                 float *S_out, float *z_out, void *workspace,
+                                 size_t workspace_bytes, kata_stream_t stream) {
+  return chunked_common(nullptr, k, v, nullptr, B, H, T, d_k, d_v, C, dtype, feature, S_out, z_out,
+                        workspace, workspace_bytes, stream, false, nullptr, nullptr, true);
 }
 
 kata_status_t kata_fwd_quadratic(const void *q, const void *k, const void *v, void *o, int B,

@@ -18,7 +18,22 @@ struct ChunkedLaunch {
   float *agg;          // per-segment increments [BH][G][D][d_v + 1]
   int G, seg_len;      // segments per head, tokens per segment
   cudaStream_t stream;
+  // initial state (library layout, nullable): the state of the tokens before
+  // this sequence, added to every segment's carry-in
+  const float *S0 = nullptr, *z0 = nullptr;
+  // only the state after the T tokens (S_out, z_out); q and o are not read
+  bool state_only = false;
 };
+
+// Sum of the G segment increments of each head, written as the state in the
+// library layout ([BH][D][d_v] and [BH][D]). The increments are in the layout
+// of the kernel that wrote them: kAggLibrary [D][d_v + 1] (z last, CUDA-core
+// kernels), kAggPsdTc (528 x 64 in the PSD tensor-core kernel's feature order
+// and scaling, then the 32 x 32 matrix sum k k^T), kAggFoTc (65 x 65: [K|1]^T
+// [V|1], minus `count_pad` padded rows from the count).
+enum AggLayout : int { kAggLibrary = 0, kAggPsdTc = 1, kAggFoTc = 2 };
+cudaError_t state_reduce(AggLayout layout, const float *agg, long long BH, int G, int D, int d_k,
+                         int d_v, float *S_out, float *z_out, float count_pad, cudaStream_t stream);
 
 struct QuadraticLaunch {
   const void *q, *k, *v;

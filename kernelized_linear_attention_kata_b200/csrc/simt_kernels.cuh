@@ -84,8 +84,8 @@ __global__ void __launch_bounds__(576) segment_increment_kernel(const Tin *__res
 }
 
 // ---------------------------------------------------------------------------
-// Pass 2: one thread block per (b, h, segment). The carry-in is the sum of
-// the increments of the earlier segments; the block then walks its chunks in
+// Pass 2: one thread block per (b, h, segment). The carry-in is the initial
+// state (if given) plus the increments of the earlier segments; the block then walks its chunks in
 // order: intra-chunk block + readout of the carried state, then the state
 // update, exactly the chunked-state recurrence.
 //
@@ -144,7 +144,8 @@ template <int DK, int DV, int FEAT, typename Tin>
 __global__ void __launch_bounds__(kSegThreads)
 segment_pass_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                     const Tin *__restrict__ v, Tin *__restrict__ o,
-                    const float *__restrict__ agg, float *__restrict__ S_out,
+                    const float *__restrict__ agg, const float *__restrict__ S0,
+                    const float *__restrict__ z0, float *__restrict__ S_out,
                     float *__restrict__ z_out, unsigned *status, int T, int C, int G,
                     int seg_len) {
   constexpr int D = state_dim(DK, FEAT);
@@ -166,12 +167,15 @@ segment_pass_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
   const int tid = threadIdx.x;
   fill_row_table<DK, FEAT>(tab, tid, kSegThreads);
 
-  // carry-in: exclusive prefix over the earlier segments' increments
+  // carry-in: the initial state (if any) plus the exclusive prefix over the
+  // earlier segments' increments
   for (int e = tid; e < D * (DV + 1); e += kSegThreads) {
+    const int r = e / (DV + 1), c = e % (DV + 1);
     float s = 0.f;
+    if (c < DV && S0) s = S0[((size_t)bh * D + r) * DV + c];
+    if (c == DV && z0) s = z0[(size_t)bh * D + r];
     const float *src = agg + (size_t)bh * G * D * (DV + 1) + e;
     for (int gp = 0; gp < g; ++gp) s += src[(size_t)gp * D * (DV + 1)];
-    const int r = e / (DV + 1), c = e % (DV + 1);
     if (c < DV) S[r * DV + c] = s;
     else z[r] = s;
   }

@@ -15,6 +15,16 @@ cudaError_t simt_chunked(const ChunkedLaunch &a) {
   const Tin *k = static_cast<const Tin *>(a.k);
   const Tin *v = static_cast<const Tin *>(a.v);
   Tin *o = static_cast<Tin *>(a.o);
+  if (a.state_only) {
+    // every segment's increment, then their sum in the library layout
+    ProfileScope prof("simt_segment_increment", a.stream);
+    segment_increment_kernel<DK, DV, FEAT, Tin><<<(unsigned)(a.BH * a.G), (D + 31) / 32 * 32, 0,
+                                                   a.stream>>>(k, v, a.agg, a.T, a.G, a.G,
+                                                               a.seg_len);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return state_reduce(kAggLibrary, a.agg, a.BH, a.G, D, DK, DV, a.S_out, a.z_out, 0.f, a.stream);
+  }
   if (a.G > 1) {
     const int threads = (D + 31) / 32 * 32;
     ProfileScope prof("simt_segment_increment", a.stream);
@@ -30,7 +40,7 @@ cudaError_t simt_chunked(const ChunkedLaunch &a) {
   if (e != cudaSuccess) return e;
   ProfileScope prof("simt_segment_pass", a.stream);
   kern<<<(unsigned)(a.BH * a.G), kSegThreads, smem, a.stream>>>(
-      q, k, v, o, a.agg, a.S_out, a.z_out, a.status, a.T, a.C, a.G, a.seg_len);
+      q, k, v, o, a.agg, a.S0, a.z0, a.S_out, a.z_out, a.status, a.T, a.C, a.G, a.seg_len);
   return cudaGetLastError();
 }
 

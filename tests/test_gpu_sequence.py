@@ -1,0 +1,129 @@
+"""GPU parity of the state-only call (kata_chunked_state) and of the forward
+from a given state (kata_fwd_chunked_from_state), the two entry points of the
+sequence-sharded forward, through the C ABI, against the fp64 oracle.
+
+A sequence cut into slices is processed slice by slice as the ranks of the
+sequence-sharded forward would: each slice's state from kata_chunked_state,
+the carry into slice r = the sum of the states of slices 0 .. r-1, each
+slice's outputs from kata_fwd_chunked_from_state. The concatenated outputs
+must match the definition on the whole sequence (per-row bound of the
+forward: 1e-4 fp32, 2e-2 bf16), and the last slice's final state the whole
+sequence's (1e-4 of the largest entry; 1e-2 for the bf16 PSD tensor-core
+path, whose update multiplies bf16-rounded key products).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from kernelized_linear_attention_kata_b200 import api
+from kernelized_linear_attention_kata_b200 import build as kbuild
+from kernelized_linear_attention_kata_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+f64 = W.to_f64_numpy
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    kbuild.build()
+    api.lib()
+
+
+def rel_rows(y, ref):
+    y = np.asarray(y, dtype=np.float64)
+    return float(np.max(np.max(np.abs(y - ref), -1) / np.maximum(np.max(np.abs(ref), -1), 1e-6)))
+
+
+def oracle_state(k, v, feature):
+    kn, vn = f64(k), f64(v)
+    B, H = kn.shape[:2]
+    D = O.state_dim(kn.shape[3], feature)
+    S = np.empty((B, H, D, vn.shape[3]))
+    z = np.empty((B, H, D))
+    for b in range(B):
+        for h in range(H):
+            S[b, h], z[b, h] = O.final_state(kn[b, h], vn[b, h], feature)
+    return S, z
+
+
+def state_tol(dtype, feature, d_k, d_v, C):
+    tc_psd = dtype == "bf16" and feature == "psd" and (d_k, d_v) == (32, 64) and C in (64, 128)
+    return 1e-2 if tc_psd else 1e-4
+
+
+# (feature, dtype, B, H, T, d_k, d_v, C, slice boundaries): the tensor-core
+# PSD and first-order paths, the CUDA-core path in fp32 and bf16, ragged
+# slices and chunk tails
+CASES = [
+    ("psd", "bf16", 1, 2, 700, 32, 64, 128, [0, 256, 300, 700]),
+    ("psd", "bf16", 2, 3, 513, 32, 64, 64, [0, 129, 513]),
+    ("first_order", "bf16", 1, 2, 600, 64, 64, 64, [0, 128, 257, 600]),
+    ("psd", "f32", 1, 2, 400, 16, 16, 64, [0, 64, 65, 400]),
+    ("psd", "bf16", 1, 1, 300, 16, 32, 32, [0, 100, 300]),
+    ("first_order", "f32", 2, 2, 333, 32, 32, 128, [0, 200, 333]),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c[:8])))
+def test_state_only_matches_oracle(case):
+    feature, dtype, B, H, T, d_k, d_v, C, _ = case
+    w = W.Workload("state", B=B, H=H, T=T, d_k=d_k, d_v=d_v, C=C, dtype=dtype, feature=feature,
+                   seed=500 + T, recipe="unit")
+    q, k, v = W.make_inputs(w)
+    S, z = api.chunked_state(k.cuda(), v.cuda(), C, feature)
+    S_ref, z_ref = oracle_state(k, v, feature)
+    tol = state_tol(dtype, feature, d_k, d_v, C)
+    assert np.max(np.abs(S.cpu().numpy() - S_ref)) <= tol * np.max(np.abs(S_ref))
+    assert np.max(np.abs(z.cpu().numpy() - z_ref)) <= tol * np.max(np.abs(z_ref))
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c[:8])))
+def test_slices_from_carried_state_match_whole_sequence(case):
+    feature, dtype, B, H, T, d_k, d_v, C, cuts = case
+    w = W.Workload("slices", B=B, H=H, T=T, d_k=d_k, d_v=d_v, C=C, dtype=dtype, feature=feature,
+                   seed=600 + T, recipe="unit")
+    q, k, v = W.make_inputs(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    D = api.state_dim(d_k, feature)
+    S0 = torch.zeros((B, H, D, d_v), dtype=torch.float32, device="cuda")
+    z0 = torch.zeros((B, H, D), dtype=torch.float32, device="cuda")
+    outs = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        sl = (slice(None), slice(None), slice(a, b))
+        qs, ks, vs = (t[sl].contiguous() for t in (qd, kd, vd))
+        o = torch.empty_like(vs)
+        S_out, z_out = torch.empty_like(S0), torch.empty_like(z0)
+        api.kata_fwd_chunked(qs, ks, vs, o, C, feature, S_out=S_out, z_out=z_out, S0=S0, z0=z0)
+        outs.append(o)
+        # the carry into the next slice, as the sequence-sharded forward forms
+        # it: the previous carry plus this slice's own state
+        Sl, zl = api.chunked_state(ks, vs, C, feature)
+        S0, z0 = S0 + Sl, z0 + zl
+        # the forward's own final state agrees with that carry
+        tol_s = state_tol(dtype, feature, d_k, d_v, C)
+        assert torch.max(torch.abs(S_out - S0)) <= tol_s * torch.max(torch.abs(S0))
+    y = torch.cat(outs, dim=2).float().cpu().numpy()
+    ref = O.per_head(O.forward_brute_force, f64(q), f64(k), f64(v), feature)
+    tol = 1e-4 if dtype == "f32" else 2e-2
+    assert rel_rows(y, ref) <= tol
+    S_ref, z_ref = oracle_state(k, v, feature)
+    tol_s = state_tol(dtype, feature, d_k, d_v, C)
+    assert np.max(np.abs(S0.cpu().numpy() - S_ref)) <= tol_s * np.max(np.abs(S_ref))
+    assert np.max(np.abs(z0.cpu().numpy() - z_ref)) <= tol_s * np.max(np.abs(z_ref))
+
+
+def test_from_state_with_no_tokens_returns_the_state():
+    D = api.state_dim(32, "psd")
+    S0 = torch.randn((1, 2, D, 64), device="cuda")
+    z0 = torch.rand((1, 2, D), device="cuda")
+    q = torch.empty((1, 2, 0, 32), device="cuda", dtype=torch.bfloat16)
+    v = torch.empty((1, 2, 0, 64), device="cuda", dtype=torch.bfloat16)
+    S_out, z_out = torch.empty_like(S0), torch.empty_like(z0)
+    api.kata_fwd_chunked(q, q, v, torch.empty_like(v), 64, "psd", S_out=S_out, z_out=z_out,
+                         S0=S0, z0=z0)
+    torch.cuda.synchronize()
+    assert torch.equal(S_out, S0) and torch.equal(z_out, z0)

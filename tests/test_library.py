@@ -119,6 +119,20 @@ def test_backward_host_checks(lib):
     assert lib.kata_bwd_chunked_workspace_bytes(-1, 1, 16, 32, 64, 64, 1, 0) == 0
 
 
+def test_state_and_from_state_host_checks(lib):
+    p = ctypes.c_void_p(256)
+    st = lib.kata_chunked_state
+    assert st(p, p, 1, 1, 16, 24, 64, 64, 1, 0, p, p, p, 1 << 20, None) == L.KATA_ERR_UNSUPPORTED
+    assert st(p, p, -1, 1, 16, 32, 64, 64, 1, 0, p, p, p, 1 << 20, None) == L.KATA_ERR_INVALID_ARGUMENT
+    assert st(p, p, 1, 1, 16, 32, 64, 0, 1, 0, p, p, p, 1 << 20, None) == L.KATA_ERR_INVALID_ARGUMENT
+    assert st(p, p, 1, 1, 16, 32, 64, 64, 1, 0, p, p, None, 1 << 20, None) == L.KATA_ERR_WORKSPACE
+    fs = lib.kata_fwd_chunked_from_state
+    assert fs(p, p, p, p, 1, 1, 16, 24, 64, 64, 1, 0, p, p, p, p, p, 1 << 20, None) == L.KATA_ERR_UNSUPPORTED
+    assert fs(p, p, p, p, 1, 1, -2, 32, 64, 64, 1, 0, p, p, p, p, p, 1 << 20, None) == L.KATA_ERR_INVALID_ARGUMENT
+    assert fs(p, p, p, p, 1, 1, 16, 32, 64, 64, 1, 0, p, p, p, p, ctypes.c_void_p(264), 1 << 20,
+              None) == L.KATA_ERR_WORKSPACE
+
+
 def test_empty_problems_launch_nothing(lib):
     p = ctypes.c_void_p(256)
     assert lib.kata_fwd_quadratic(p, p, p, p, 0, 4, 8, 32, 64, 1, 0, None) == L.KATA_OK

@@ -1,7 +1,10 @@
-"""The benchmark's multi-rank host logic on CPU, with world_size-2 gloo ranks:
-every rank learns the slowest rank's step time, the whole-job throughput
-counts every rank's tokens, and the reference arm runs on rank 0 only.
-(The data path itself has no collective: ranks are independent replicas.)"""
+"""Multi-rank host logic on CPU, with gloo ranks:
+
+* the benchmark: every rank learns the slowest rank's step time, the
+  whole-job throughput counts every rank's tokens, and the reference arm runs
+  on rank 0 only (head-sharded replicas have no data-path collective);
+* the sequence-sharded forward's one exchange: rank r receives the sum of
+  the states of ranks 0 .. r-1 (the carry into its slice)."""
 
 import os
 import socket
@@ -67,3 +70,38 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
 
     assert bench.run_reference(Args, 1, 2) == 0     # rank 1: no work, no output
     assert capsys.readouterr().out == ""
+
+
+def _prefix_main(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import torch
+
+        from kernelized_linear_attention_kata_b200.sequence_parallel import \
+            exclusive_prefix_over_ranks
+        # rank r's "state": distinct powers of two, so every partial sum is exact
+        # and identifies exactly which ranks were summed
+        local = torch.full((3, 5), float(2 ** rank), dtype=torch.float32)
+        local[0, 0] = float(rank + 1) * 1000.0
+        out[rank] = exclusive_prefix_over_ranks(local).tolist()
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_shards_receive_the_exclusive_prefix(world):
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_prefix_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    for rank in range(world):
+        got = res[rank]
+        want_fill = float(sum(2 ** r for r in range(rank)))
+        want_corner = float(sum((r + 1) * 1000 for r in range(rank)))
+        assert got[0][0] == want_corner
+        assert all(x == want_fill for row in got for x in row[1:])
+        assert all(row[0] == want_fill for row in got[1:])
