@@ -303,7 +303,11 @@ def run_ours(args, rank, world, local_rank):
     elif args.T:
         w = w.with_T(args.T)
     from dataclasses import replace
-    w = replace(w, seed=w.seed + 1000 * rank)     # one seeded batch per rank
+    seq = args.shard == "sequence"
+    if seq and (form != "chunked" or w.T % world):
+        raise SystemExit("--shard sequence needs --form chunked and T divisible by the ranks")
+    if not seq:
+        w = replace(w, seed=w.seed + 1000 * rank)     # one seeded batch per rank
     stream = torch.cuda.current_stream()
     if form == "decode":
         B, H = args.decode_batch, W.DECODE_HEADS
@@ -345,12 +349,25 @@ def run_ours(args, rank, world, local_rank):
                 api.kata_fwd_quadratic(q, k, v, o, w.feature)
             flops_th = (w.T + 1) / 2 * (2 * w.d_k + 2 * w.d_v + 2)
             _, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
-        else:
-            ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
-            seq = form == "sequential"
+        elif seq:
+            # one sequence cut along T, this rank's slice of it
+            from kernelized_linear_attention_kata_b200 import sequence_parallel as SP
+            Tr = w.T // world
+            sl = (slice(None), slice(None), slice(rank * Tr, (rank + 1) * Tr))
+            q, k, v = (t[sl].contiguous() for t in (q, k, v))
+            o = torch.empty_like(v)
+            w = w.with_T(Tr)
+            ws = None
 
             def step():
-                api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws, sequential=seq)
+                SP.fwd_chunked_sequence_parallel(q, k, v, w.C, w.feature, out=o)
+            flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
+        else:
+            ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
+            seq_carry = form == "sequential"
+
+            def step():
+                api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws, sequential=seq_carry)
             flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
         tokens_per_step = w.B * w.T
         token_heads = w.B * w.H * w.T
@@ -468,9 +485,9 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         line = {
             "metric": METRIC_BWD if form == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong" if seq else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": config | {"parallelism": f"replicas x{world}"},
+            "config": config | {"parallelism": f"sequence x{world}" if seq else f"replicas x{world}"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
             "kernels": {n: {"launches": c, "avg_ms": t / c} for n, (c, t) in prof.items()},
             "clocks": clocks.summary(), "token_heads_per_s": value * token_heads / tokens_per_step,
@@ -489,6 +506,10 @@ def main():
     ap.add_argument("--form", default="chunked",
                     choices=["chunked", "sequential", "first_order", "quadratic", "decode", "backward"],
                     help="chunked is the headline; the others are secondary measurements")
+    ap.add_argument("--shard", choices=["heads", "sequence"], default="heads",
+                    help="heads: independent replicas, one batch per rank (weak scaling); "
+                         "sequence: one sequence cut along T, one slice per rank, one all-reduce "
+                         "of the slice states (strong scaling)")
     ap.add_argument("--decode-batch", type=int, default=W_DECODE_BATCH)
     ap.add_argument("--T", type=int, default=0, help="override T (profiling a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")

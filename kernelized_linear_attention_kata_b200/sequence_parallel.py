@@ -28,7 +28,10 @@ from . import api
 
 def exclusive_prefix_over_ranks(flat: torch.Tensor, group=None) -> torch.Tensor:
     """Sum of the ranks' `flat` tensors over the ranks before this one
-    (zeros on rank 0), by one all-reduce of a [world, n] buffer."""
+    (zeros on rank 0), by one all-reduce of a [world, n] buffer. Without a
+    process group there is one rank, and the carry is zero."""
+    if not dist.is_initialized():
+        return torch.zeros_like(flat)
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     buf = torch.zeros((world, flat.numel()), dtype=flat.dtype, device=flat.device)
@@ -37,16 +40,18 @@ def exclusive_prefix_over_ranks(flat: torch.Tensor, group=None) -> torch.Tensor:
     return buf[rank].reshape(flat.shape)
 
 
-def fwd_chunked_sequence_parallel(q, k, v, C, feature="psd", group=None, return_state=False):
+def fwd_chunked_sequence_parallel(q, k, v, C, feature="psd", group=None, return_state=False,
+                                  out=None):
     """This rank's outputs for its slice q, k, v [B, H, T_r, d] of a sequence
-    cut along T in rank order. With return_state, also the state after the
-    slice (on the last rank: the state of the whole sequence)."""
+    cut along T in rank order (into `out` if given). With return_state, also
+    the state after the slice (on the last rank: the state of the whole
+    sequence)."""
     S_loc, z_loc = api.chunked_state(k, v, C, feature)
     nS = S_loc.numel()
     carry = exclusive_prefix_over_ranks(torch.cat([S_loc.reshape(-1), z_loc.reshape(-1)]), group)
     S0 = carry[:nS].view_as(S_loc)
     z0 = carry[nS:].view_as(z_loc)
-    o = torch.empty_like(v)
+    o = torch.empty_like(v) if out is None else out
     if return_state:
         S_out, z_out = torch.empty_like(S_loc), torch.empty_like(z_loc)
         api.kata_fwd_chunked(q, k, v, o, C, feature, S_out=S_out, z_out=z_out, S0=S0, z0=z0)

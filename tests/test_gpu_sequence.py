@@ -127,3 +127,15 @@ def test_from_state_with_no_tokens_returns_the_state():
                          S0=S0, z0=z0)
     torch.cuda.synchronize()
     assert torch.equal(S_out, S0) and torch.equal(z_out, z0)
+
+
+def test_sequence_parallel_on_one_rank_is_the_plain_forward():
+    """Without a process group there is one slice and a zero carry."""
+    from kernelized_linear_attention_kata_b200 import sequence_parallel as SP
+    w = W.Workload("sp1", B=1, H=2, T=300, d_k=32, d_v=64, C=128, dtype="bf16", feature="psd",
+                   seed=71, recipe="unit")
+    q, k, v = (t.cuda() for t in W.make_inputs(w))
+    o_sp, S_sp, z_sp = SP.fwd_chunked_sequence_parallel(q, k, v, w.C, w.feature, return_state=True)
+    o, S, z = api.fwd_chunked(q, k, v, w.C, w.feature, return_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_sp, o) and torch.equal(S_sp, S) and torch.equal(z_sp, z)
