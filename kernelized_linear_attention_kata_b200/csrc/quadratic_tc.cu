@@ -14,8 +14,12 @@
 // Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM
 // and issues MMAs (one elected lane), warps 2-5 are the math warps; math
 // thread r owns TMEM lane r = query row r of the block.
-// TMEM: S_j in columns [0, 128) (P_j packed bf16 overwrites [0, 64)),
-// O in [128, 192). 256 columns are allocated, so two CTAs share an SM.
+// Each key block is processed as two 64-key halves with their own barriers:
+// S of half 0 in TMEM columns [0, 64), of half 1 in [64, 128), each half's P
+// packed as bf16 over its first 32 columns; O in [128, 192). The math warps
+// square one half while the tensor pipe runs P V of the other half and Q K^T
+// of the next block's same half. 256 columns are allocated, so two CTAs
+// share an SM.
 #include "common.cuh"
 #include "launch.h"
 #include "profile.h"
@@ -28,6 +32,7 @@ namespace {
 using namespace tc;
 
 constexpr int kBlock = 128;       // queries per CTA, keys per block
+constexpr int kHalf = 64;         // keys per half block (one S buffer)
 constexpr int kDV = 64;
 constexpr int kStages = 2;
 constexpr int kThreads = 192;
@@ -43,8 +48,8 @@ struct QuadLayout {
   static constexpr int kK = kQ + kQKBytes;
   static constexpr int kV = kK + kStages * kQKBytes;
   static constexpr int kBar = kV + kStages * kVBytes;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full, p_full, o_full
-  static constexpr int kNumBars = 4 + 2 * kStages;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full
+  static constexpr int kNumBars = 6 + 2 * kStages;
   static constexpr int kTmemSlot = kBar + 8 * kNumBars;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kBytes = kAbort + 4;
@@ -65,9 +70,9 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   uint64_t *q_full = bars;
   uint64_t *kv_full = bars + 1;
   uint64_t *kv_empty = bars + 1 + kStages;
-  uint64_t *s_full = bars + 1 + 2 * kStages;
-  uint64_t *p_full = s_full + 1;
-  uint64_t *o_full = s_full + 2;
+  uint64_t *s_full = bars + 1 + 2 * kStages;     // [2]: one per 64-key half
+  uint64_t *p_full = s_full + 2;                 // [2]
+  uint64_t *o_full = s_full + 4;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kAbort);
 
@@ -83,8 +88,10 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&s_full[h], 1);
+      mbar_init(&p_full[h], 128);
+    }
     mbar_init(o_full, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -116,44 +123,53 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // Each 128-key block is handled as two 64-key halves with their own
+    // barriers, so that the math warps square one half while the tensor pipe
+    // runs P V of the other and Q K^T of the next block's same half (issued
+    // after that P V, which has then read the half's P: the pipe runs MMAs
+    // in order).
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(kBlock, kBlock, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16(kBlock, kHalf, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(kBlock, kDV, false, true);
       const uint32_t q_addr = smem_u32(smem + L::kQ);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      for (int j = 0; ok && j < nkb; ++j) {
-        const int s = j % kStages;
-        if (j > 0) {
-          const int sp = (j - 1) % kStages;
-          if (!(ok = mbar_wait(p_full, (j - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(smem + L::kV + sp * L::kVBytes);
-#pragma unroll
-          for (int kk = 0; kk < kBlock / 16; ++kk)
-            mma_ts(tbase + kColO, tbase + kColS + 8 * kk,
-                   smem_desc(v_addr + kk * 2048, 16384, 1024, kSw128), idesc_pv,
-                   (j - 1 > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&kv_empty[sp]);
-        }
-        if (!(ok = mbar_wait(&kv_full[s], (j / kStages) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + L::kK + s * L::kQKBytes);
+      auto issue_qk = [&](int j, int h) {
+        const uint32_t k_addr = smem_u32(smem + L::kK + (j % kStages) * L::kQKBytes) +
+                                (uint32_t)(h * kHalf * L::kRowBytes);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
-          mma_ss(tbase + kColS, smem_desc(q_addr + kk * 32, 16, 8 * L::kRowBytes, L::kSwizzle),
+          mma_ss(tbase + kColS + kHalf * h, smem_desc(q_addr + kk * 32, 16, 8 * L::kRowBytes, L::kSwizzle),
                  smem_desc(k_addr + kk * 32, 16, 8 * L::kRowBytes, L::kSwizzle), idesc_qk,
                  kk > 0 ? 1u : 0u);
-        mma_commit(s_full);
-      }
-      if (ok && mbar_wait(p_full, (nkb - 1) & 1, abort_flag)) {
+        mma_commit(&s_full[h]);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
+      if (ok) {
         tc_fence_after();
-        const int sp = (nkb - 1) % kStages;
-        const uint32_t v_addr = smem_u32(smem + L::kV + sp * L::kVBytes);
+        issue_qk(0, 0);
+        issue_qk(0, 1);
+      }
+      for (int j = 0; ok && j < nkb; ++j) {
+        const int s = j % kStages;
+        const uint32_t v_addr = smem_u32(smem + L::kV + s * L::kVBytes);
+        for (int h = 0; ok && h < 2; ++h) {
+          if (!(ok = mbar_wait(&p_full[h], j & 1, abort_flag))) break;
+          tc_fence_after();
+          // O += P_h V_h (P_h: 64 keys as 32 packed columns of tensor memory)
 #pragma unroll
-        for (int kk = 0; kk < kBlock / 16; ++kk)
-          mma_ts(tbase + kColO, tbase + kColS + 8 * kk,
-                 smem_desc(v_addr + kk * 2048, 16384, 1024, kSw128), idesc_pv,
-                 (nkb - 1 > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kHalf / 16; ++kk)
+            mma_ts(tbase + kColO, tbase + kColS + kHalf * h + 8 * kk,
+                   smem_desc(v_addr + (4 * h + kk) * 2048, 16384, 1024, kSw128), idesc_pv,
+                   (j > 0 || h > 0 || kk > 0) ? 1u : 0u);
+          if (h == 1) mma_commit(&kv_empty[s]);        // K_j, V_j no longer read
+          if (j + 1 < nkb) {
+            if (h == 0) {
+              if (!(ok = mbar_wait(&kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, abort_flag)))
+                break;
+              tc_fence_after();
+            }
+            issue_qk(j + 1, h);
+          }
+        }
       }
       mma_commit(o_full);
     }
@@ -167,45 +183,47 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
     bool ok = true;
-    for (int j = 0; j < nkb; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, j & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const int key0 = j * kBlock;
+    for (int j = 0; ok && j < nkb; ++j) {
       // key blocks below the diagonal block lie entirely before every query
       // of this block (and before T): no mask there
       const bool diag = j == nkb - 1;
+      for (int h = 0; h < 2; ++h) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[h], j & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const int key0 = j * kBlock + kHalf * h;
 #pragma unroll 1
-      for (int c = 0; c < kBlock / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tbase + lane_off + kColS + 32 * c, r);
-        tmem_wait_ld();
-        uint32_t p[16];
-        if (!diag) {
+        for (int c = 0; c < kHalf / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + lane_off + kColS + kHalf * h + 32 * c, r);
+          tmem_wait_ld();
+          uint32_t p[16];
+          if (!diag) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 x = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            const float2 w = FEAT == kPSD ? __fmul2_rn(x, x) : __fadd2_rn(make_float2(1.f, 1.f), x);
-            lsum[i & 3] = __fadd2_rn(lsum[i & 3], w);
-            p[i] = pack_bf16x2(w.x, w.y);
-          }
-        } else {
+            for (int i = 0; i < 16; ++i) {
+              const float2 x = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              const float2 w = FEAT == kPSD ? __fmul2_rn(x, x) : __fadd2_rn(make_float2(1.f, 1.f), x);
+              lsum[i & 3] = __fadd2_rn(lsum[i & 3], w);
+              p[i] = pack_bf16x2(w.x, w.y);
+            }
+          } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int k0 = key0 + 32 * c + 2 * i;
-            const float2 x = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            float2 w = FEAT == kPSD ? __fmul2_rn(x, x) : __fadd2_rn(make_float2(1.f, 1.f), x);
-            if (k0 > t || k0 >= T) w.x = 0.f;
-            if (k0 + 1 > t || k0 + 1 >= T) w.y = 0.f;
-            lsum[i & 3] = __fadd2_rn(lsum[i & 3], w);
-            p[i] = pack_bf16x2(w.x, w.y);
+            for (int i = 0; i < 16; ++i) {
+              const int k0 = key0 + 32 * c + 2 * i;
+              const float2 x = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              float2 w = FEAT == kPSD ? __fmul2_rn(x, x) : __fadd2_rn(make_float2(1.f, 1.f), x);
+              if (k0 > t || k0 >= T) w.x = 0.f;
+              if (k0 + 1 > t || k0 + 1 >= T) w.y = 0.f;
+              lsum[i & 3] = __fadd2_rn(lsum[i & 3], w);
+              p[i] = pack_bf16x2(w.x, w.y);
+            }
           }
+          tmem_st16(tbase + lane_off + kColS + kHalf * h + 16 * c, p);
         }
-        tmem_st16(tbase + lane_off + kColS + 16 * c, p);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[h]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
     }
     const float2 l01 = __fadd2_rn(lsum[0], lsum[1]), l23 = __fadd2_rn(lsum[2], lsum[3]);
     const float l = (l01.x + l01.y) + (l23.x + l23.y);

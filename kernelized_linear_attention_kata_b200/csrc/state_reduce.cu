@@ -27,12 +27,14 @@ __device__ __forceinline__ int psd_tc_feature(int i, int j) {
 __global__ void __launch_bounds__(kReduceThreads)
 state_reduce_kernel(int layout, const float *__restrict__ agg, int G, int D, int d_k, int d_v,
                     float *__restrict__ S_out, float *__restrict__ z_out, float count_pad) {
-  const int bh = blockIdx.x;
+  const int nb = (D * (d_v + 1) + kReduceThreads - 1) / kReduceThreads;   // blocks per head
+  const long long bh = blockIdx.x / nb;
   const size_t inc = layout == kAggLibrary ? (size_t)D * (d_v + 1)
                    : layout == kAggPsdTc   ? (size_t)D * d_v + (size_t)d_k * d_k
                                            : (size_t)(d_k + 1) * (d_k + 1);
   const float *base = agg + (size_t)bh * G * inc;
-  for (int e = threadIdx.x; e < D * (d_v + 1); e += kReduceThreads) {
+  const int e = (int)(blockIdx.x % nb) * kReduceThreads + threadIdx.x;   // one state entry per thread
+  if (e < D * (d_v + 1)) {
     const int r = e / (d_v + 1), c = e % (d_v + 1);     // library row r, column c (c = d_v: z)
     size_t off;
     float scale = 1.f, pad = 0.f;
@@ -70,8 +72,10 @@ state_reduce_kernel(int layout, const float *__restrict__ agg, int G, int D, int
 cudaError_t state_reduce(AggLayout layout, const float *agg, long long BH, int G, int D, int d_k,
                          int d_v, float *S_out, float *z_out, float count_pad, cudaStream_t stream) {
   ProfileScope prof("state_reduce", stream);
-  state_reduce_kernel<<<(unsigned)BH, kReduceThreads, 0, stream>>>((int)layout, agg, G, D, d_k, d_v,
-                                                                   S_out, z_out, count_pad);
+  const long long nb = (D * (d_v + 1) + kReduceThreads - 1) / kReduceThreads;
+  state_reduce_kernel<<<(unsigned)(BH * nb), kReduceThreads, 0, stream>>>((int)layout, agg, G, D, d_k,
+                                                                          d_v, S_out, z_out,
+                                                                          count_pad);
   return cudaGetLastError();
 }
 
