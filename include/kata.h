@@ -41,6 +41,11 @@
  *    records this in its workspace; see kata_workspace_status.
  *  - B, H or T equal to 0 is a valid empty problem: nothing is launched for
  *    the outputs (S_out / z_out, when given, are zero-filled).
+ *  - Reproducibility: the states are bitwise reproducible. The bf16
+ *    tensor-core chunked forward for PSD (d_k = 32, d_v = 64) accumulates its
+ *    readout from two MMA-issuing threads into one fp32 accumulator, in an
+ *    order that varies from run to run, so its outputs can differ between
+ *    runs in the last bf16 bit.
  *
  * Supported shapes (anything else returns KATA_ERR_UNSUPPORTED):
  *    PSD          d_k in {16, 32}

@@ -591,57 +591,64 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         uint32_t R[32];
 #pragma unroll
         for (int l = 0; l < 32; ++l) R[l] = P[l];
-#pragma unroll 1
-        for (int s9 = 0; s9 < kQSlots; ++s9) {
+        // Entry ring_entry(s9) may be written once its previous use has been
+        // read. The first use of a chunk of a tensor-memory entry instead
+        // waits for what last used the columns in this chunk (P V for entries
+        // 1 and 2, U for entry 3), which also implies every use of the
+        // previous chunk is complete; entry 3 first hands its U to the
+        // denominator.
+        auto wait_entry = [&](int s9) -> bool {
           const int b = ring_entry(s9), j = s9 / kRing, k = ring_uses(b) * i + j;
-          // Entry b may be written once its previous use has been read. The
-          // first use of a chunk of a tensor-memory entry instead waits for
-          // what last used the columns in this chunk (P V for entries 1 and
-          // 2, U for entry 3), which also implies every use of the previous
-          // chunk is complete; entry 3 first hands its U to the denominator.
-          if (ok) {
-            if (j == 0 && b == 1) {
-              ok = warp_wait(&bars[kBarPVDone], i & 1, abort_flag);
-            } else if (j == 0 && b == 2) {
-              // P V already waited for (entry 1 comes first)
-            } else if (j == 0 && b == 3) {
-              ok = warp_wait(&bars[kBarUDone], i & 1, abort_flag);
-              if (ok) {
-                tc_fence_after();
-                uint32_t uu[32];
-                tmem_ld32(tbase + lane_off + kColU, uu);
-                tmem_wait_ld();
-#pragma unroll
-                for (int w = 0; w < 16; ++w) {
-                  const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162 *>(&XQ[w]);
-                  den_inter = fmaf(__low2float(qq), __uint_as_float(uu[2 * w]), den_inter);
-                  den_inter = fmaf(__high2float(qq), __uint_as_float(uu[2 * w + 1]), den_inter);
-                }
-              }
-            } else if (k > 0) {
-              ok = warp_wait(&bars[kBarRingEmpty + b], (k - 1) & 1, abort_flag);
-            }
-          }
-          // the slot is read against snapshot tile s9 / 2 of S_c
-          if (ok && (s9 & 1) == 0) ok = warp_wait(&bars[kBarTileSnap + (s9 >> 1)], i & 1, abort_flag);
-          if (ok) {
+          if (j == 0 && b == 1) return warp_wait(&bars[kBarPVDone], i & 1, abort_flag);
+          if (j == 0 && b == 2) return true;             // P V already waited for (entry 1 first)
+          if (j == 0 && b == 3) {
+            if (!warp_wait(&bars[kBarUDone], i & 1, abort_flag)) return false;
             tc_fence_after();
-            uint32_t w[32];
-            q_slot_words(P, R, s9 == kQSlots - 1, w);
-            if (b == 0) {
+            uint32_t uu[32];
+            tmem_ld32(tbase + lane_off + kColU, uu);
+            tmem_wait_ld();
 #pragma unroll
-              for (int cc = 0; cc < 8; ++cc)
-                *reinterpret_cast<uint4 *>(qslot + sw128(r, cc)) =
-                    make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
-              fence_async_smem();
-            } else {
-              tmem_st32(tbase + lane_off + ring_col(b), w);
-              tmem_wait_st();
-              tc_fence_before();
+            for (int w = 0; w < 16; ++w) {
+              const __nv_bfloat162 qq = *reinterpret_cast<const __nv_bfloat162 *>(&XQ[w]);
+              den_inter = fmaf(__low2float(qq), __uint_as_float(uu[2 * w]), den_inter);
+              den_inter = fmaf(__high2float(qq), __uint_as_float(uu[2 * w + 1]), den_inter);
             }
-            warp_arrive(&bars[kBarRingFull + b]);
+            return true;
           }
+          return k == 0 || warp_wait(&bars[kBarRingEmpty + b], (k - 1) & 1, abort_flag);
+        };
+        // Query features of slot s9 (R rotated to its offsets) into its entry.
+        auto produce = [&](int s9) {
+          const int b = ring_entry(s9);
+          tc_fence_after();
+          uint32_t w[32];
+          q_slot_words(P, R, s9 == kQSlots - 1, w);
+          if (b == 0) {
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+              *reinterpret_cast<uint4 *>(qslot + sw128(r, cc)) =
+                  make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+            fence_async_smem();
+          } else {
+            tmem_st32(tbase + lane_off + ring_col(b), w);
+            tmem_wait_st();
+            tc_fence_before();
+          }
+          warp_arrive(&bars[kBarRingFull + b]);
+        };
+        // Slots go in pairs (2 p, 2 p + 1): one for each readout issuer, both
+        // read against snapshot tile p. The pair's waits come first, so the
+        // two issuers receive their slots together.
+#pragma unroll 1
+        for (int s9 = 0; s9 < kQSlots; s9 += 2) {
+          const bool pair = s9 + 1 < kQSlots;
+          if (ok) ok = wait_entry(s9);
+          if (ok && pair) ok = wait_entry(s9 + 1);
+          if (ok) ok = warp_wait(&bars[kBarTileSnap + (s9 >> 1)], i & 1, abort_flag);
+          if (ok) produce(s9);
           rotate_left(R, 2);
+          if (ok && pair) produce(s9 + 1);
+          if (pair) rotate_left(R, 2);
         }
         if (!ok) break;
 

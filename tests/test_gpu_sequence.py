@@ -130,7 +130,10 @@ def test_from_state_with_no_tokens_returns_the_state():
 
 
 def test_sequence_parallel_on_one_rank_is_the_plain_forward():
-    """Without a process group there is one slice and a zero carry."""
+    """Without a process group there is one slice and a zero carry. The state
+    (one MMA issuer) is bitwise the plain forward's; the outputs agree to
+    rounding: two issuers accumulate the readout into one accumulator, in an
+    order that varies from run to run."""
     from kernelized_linear_attention_kata_b200 import sequence_parallel as SP
     w = W.Workload("sp1", B=1, H=2, T=300, d_k=32, d_v=64, C=128, dtype="bf16", feature="psd",
                    seed=71, recipe="unit")
@@ -138,4 +141,7 @@ def test_sequence_parallel_on_one_rank_is_the_plain_forward():
     o_sp, S_sp, z_sp = SP.fwd_chunked_sequence_parallel(q, k, v, w.C, w.feature, return_state=True)
     o, S, z = api.fwd_chunked(q, k, v, w.C, w.feature, return_state=True)
     torch.cuda.synchronize()
-    assert torch.equal(o_sp, o) and torch.equal(S_sp, S) and torch.equal(z_sp, z)
+    assert torch.equal(S_sp, S) and torch.equal(z_sp, z)
+    a, b = o_sp.float(), o.float()
+    row_err = (a - b).abs().amax(-1) / b.abs().amax(-1).clamp_min(1e-6)
+    assert float(row_err.max()) <= 8e-3          # two bf16 rounding steps
