@@ -34,13 +34,18 @@ using namespace tc;
 constexpr int kBlock = 128;       // queries per CTA, keys per block
 constexpr int kHalf = 64;         // keys per half block (one S buffer)
 constexpr int kDV = 64;
-constexpr int kStages = 2;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColO = 128;
 
 template <int DK>
 struct QuadLayout {
+  // K, V ring depth. A block's loads are issued when the block kStages
+  // earlier has been consumed; with two stages that left about half a block
+  // of math to cover the load latency and the MMA warp waited on it every
+  // block. Four stages fit beside a second CTA on the SM for d_k <= 32;
+  // at d_k = 64 a third stage would not, so it keeps two CTAs and two stages.
+  static constexpr int kStages = DK <= 32 ? 4 : 2;
   static constexpr int kRowBytes = DK * 2;
   static constexpr int kQKBytes = kBlock * kRowBytes;     // one Q or K tile
   static constexpr int kVBytes = kBlock * kDV * 2;        // one V tile (16 KB)
@@ -69,8 +74,8 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
   uint64_t *q_full = bars;
   uint64_t *kv_full = bars + 1;
-  uint64_t *kv_empty = bars + 1 + kStages;
-  uint64_t *s_full = bars + 1 + 2 * kStages;     // [2]: one per 64-key half
+  uint64_t *kv_empty = bars + 1 + L::kStages;
+  uint64_t *s_full = bars + 1 + 2 * L::kStages;     // [2]: one per 64-key half
   uint64_t *p_full = s_full + 2;                 // [2]
   uint64_t *o_full = s_full + 4;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
@@ -84,7 +89,7 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
@@ -114,8 +119,8 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       mbar_arrive_expect_tx(q_full, L::kQKBytes);
       tma_load_3d(smem + L::kQ, &tmq, q_full, 0, qb * kBlock, bh);
       for (int j = 0; j < nkb; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages && !mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, abort_flag)) break;
+        const int s = j % L::kStages;
+        if (j >= L::kStages && !mbar_wait(&kv_empty[s], ((j / L::kStages) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&kv_full[s], L::kQKBytes + L::kVBytes);
         tma_load_3d(smem + L::kK + s * L::kQKBytes, &tmk, &kv_full[s], 0, j * kBlock, bh);
         tma_load_3d(smem + L::kV + s * L::kVBytes, &tmv, &kv_full[s], 0, j * kBlock, bh);
@@ -133,7 +138,7 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       constexpr uint32_t idesc_pv = idesc_bf16(kBlock, kDV, false, true);
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       auto issue_qk = [&](int j, int h) {
-        const uint32_t k_addr = smem_u32(smem + L::kK + (j % kStages) * L::kQKBytes) +
+        const uint32_t k_addr = smem_u32(smem + L::kK + (j % L::kStages) * L::kQKBytes) +
                                 (uint32_t)(h * kHalf * L::kRowBytes);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk)
@@ -149,7 +154,7 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
         issue_qk(0, 1);
       }
       for (int j = 0; ok && j < nkb; ++j) {
-        const int s = j % kStages;
+        const int s = j % L::kStages;
         const uint32_t v_addr = smem_u32(smem + L::kV + s * L::kVBytes);
         for (int h = 0; ok && h < 2; ++h) {
           if (!(ok = mbar_wait(&p_full[h], j & 1, abort_flag))) break;
@@ -163,7 +168,7 @@ quadratic_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           if (h == 1) mma_commit(&kv_empty[s]);        // K_j, V_j no longer read
           if (j + 1 < nkb) {
             if (h == 0) {
-              if (!(ok = mbar_wait(&kv_full[(j + 1) % kStages], ((j + 1) / kStages) & 1, abort_flag)))
+              if (!(ok = mbar_wait(&kv_full[(j + 1) % L::kStages], ((j + 1) / L::kStages) & 1, abort_flag)))
                 break;
               tc_fence_after();
             }
