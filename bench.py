@@ -61,6 +61,16 @@ def algorithmic_per_token_head(d_k, d_v, C, feature="psd"):
     return intra + update + readout, (2 * d_k + d_v) * 2 + d_v * 2
 
 
+def feature_products_per_token_head(d_k, feature="psd"):
+    """Scalar products the feature expansion needs per token-head: phi(k) for
+    the state update and phi~(q) for the readout, one product per packed
+    feature each (the query's multiplicity 2 folds into its product). The
+    first-order feature [1, u] is the input itself and needs none."""
+    if feature != "psd":
+        return 0
+    return 2 * (d_k * (d_k + 1) // 2)
+
+
 def algorithmic_backward_per_token_head(d_k, d_v, C, feature="psd"):
     """(flops, bytes) the gradient of the chunked forward must do per
     token-head: the carried parts of dq (S g + z c, then the query feature's
@@ -309,6 +319,7 @@ def run_ours(args, rank, world, local_rank):
     if not seq:
         w = replace(w, seed=w.seed + 1000 * rank)     # one seeded batch per rank
     stream = torch.cuda.current_stream()
+    phi_th = 0            # feature-expansion products per token-head, where the form has them
     if form == "decode":
         B, H = args.decode_batch, W.DECODE_HEADS
         q, k, v = W.make_decode_inputs(B, H, device=dev)
@@ -326,6 +337,7 @@ def run_ours(args, rank, world, local_rank):
         D = api.state_dim(W.DECODE_DK)
         flops_th = 2 * D * W.DECODE_DV * 2 + 3 * D
         bytes_th = 2 * 4 * D * (W.DECODE_DV + 1) + 2 * (2 * W.DECODE_DK + 2 * W.DECODE_DV)
+        phi_th = feature_products_per_token_head(W.DECODE_DK)
         config = {"workload": f"decode_b{B}_h{H}", "B": B, "H": H, "d_k": W.DECODE_DK,
                   "d_v": W.DECODE_DV, "feature": "psd", "form": "decode step",
                   "l2": "state larger than L2 (no flush needed)"}
@@ -362,6 +374,7 @@ def run_ours(args, rank, world, local_rank):
             def step():
                 SP.fwd_chunked_sequence_parallel(q, k, v, w.C, w.feature, out=o)
             flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
+            phi_th = feature_products_per_token_head(w.d_k, w.feature)
         else:
             ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
             seq_carry = form == "sequential"
@@ -369,6 +382,7 @@ def run_ours(args, rank, world, local_rank):
             def step():
                 api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws, sequential=seq_carry)
             flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
+            phi_th = feature_products_per_token_head(w.d_k, w.feature)
         tokens_per_step = w.B * w.T
         token_heads = w.B * w.H * w.T
         config = workload_config(w)
@@ -441,6 +455,13 @@ def run_ours(args, rank, world, local_rank):
     t_tensor = flops_th * token_heads / (peaks["bf16_tflops"] * 1e12)
     t_hbm = bytes_th * token_heads / (peaks["hbm_gbs"] * 1e9)
     roofline["step_frac_of_tensor_or_hbm"] = max(t_tensor, t_hbm) / (ms / 1e3)
+    # third floor: the feature expansion's products on the FP32 lanes
+    if phi_th:
+        lanes_per_s = 148 * 128 * peaks["sm_max_mhz"] * 1e6
+        floor_s = phi_th * token_heads / lanes_per_s
+        roofline["phi_alu"] = {"products_per_token_head": phi_th, "floor_ms": floor_s * 1e3,
+                               "frac_of_step": floor_s / (ms / 1e3),
+                               "peak_kind": "derived: 148 SMs x 128 FP32 lanes x max SM clock"}
     gpu_launches = sum(n for n, _ in prof.values())
 
     # end to end through the public API with pinned host buffers
