@@ -22,6 +22,11 @@ Parity status per function (what pins it is listed in tests/test_oracle_pins.py)
   fixture, forms agreement), but the READING that this is the pages'
   "first-order feature" is not fixed by the pages: parity of that reading is
   unpinned.
+* KATA-Mg, KATA-Sigma-g and DeltaKATA (oracle/variants.py) -- the pages only
+  name them; the arithmetic of each reading is pinned
+  (tests/test_oracle_variants.py: reductions to the rank-one oracle, closed
+  forms, invariances, an unpacked delta rule), parity of the readings is
+  unpinned.
 """
 
 from .kata import *  # noqa: F401,F403
@@ -33,3 +38,4 @@ from .kata import (  # noqa: F401
     psd_pairs, psd_query_feature, query_feature, state_dim, weights,
 )
 from .backward import backward_brute_force, backward_rows  # noqa: F401
+from . import variants  # noqa: F401
