@@ -72,12 +72,12 @@ def alloc_workspace(B, H, T, d_k, d_v, C, dtype=torch.bfloat16, feature="psd", d
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def _shapes(q, k, v, o):
+def _shapes(q, k, v, o, o_name="o"):
     if q.dim() != 4 or k.shape != q.shape or v.dim() != 4 or v.shape[:3] != q.shape[:3]:
         raise ValueError(f"expected q, k [B,H,T,d_k] and v [B,H,T,d_v]; got {tuple(q.shape)}, "
                          f"{tuple(k.shape)}, {tuple(v.shape)}")
     if o.shape != v.shape or o.dtype != q.dtype:
-        raise ValueError("o must have v's shape and q's dtype")
+        raise ValueError(f"{o_name} must have v's shape and q's dtype")
     if not (k.dtype == v.dtype == q.dtype):
         raise TypeError("q, k, v must share one dtype")
     B, H, T, d_k = q.shape
@@ -173,7 +173,7 @@ def bwd_chunked_workspace_bytes(B, H, T, d_k, d_v, C, dtype=torch.bfloat16, feat
 
 def kata_bwd_chunked(q, k, v, dout, dq, dk, dv, C, feature="psd", workspace=None, stream=None):
     """Gradient of the chunked forward into dq, dk, dv (see include/kata.h)."""
-    B, H, T, d_k, d_v = _shapes(q, k, v, dout)
+    B, H, T, d_k, d_v = _shapes(q, k, v, dout, "dout")
     if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
         raise ValueError("dq, dk, dv must have the shapes of q, k, v")
     for t, name in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
