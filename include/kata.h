@@ -290,12 +290,32 @@ KATA_API kata_status_t kata_bwd_chunked(const void *q, const void *k, const void
 
 /*
  * Synchronises `stream`, then reads the status word a kata_fwd_chunked(...),
- * kata_fwd_chunked_sequential(...) or kata_bwd_chunked(...) call left in
- * `workspace`: KATA_OK, or
+ * kata_fwd_chunked_sequential(...), kata_fwd_chunked_from_state(...),
+ * kata_chunked_state(...), kata_bwd_chunked(...) or
+ * kata_selftest_device_timeout(...) call left in `workspace`: KATA_OK, or
+ * KATA_ERR_DEVICE_TIMEOUT if a bounded wait inside a kernel gave up (the
+ * kernel returned early, its outputs are undefined, the context is usable),
  * KATA_ERR_NONPOSITIVE_NORMALISER if any row had a normaliser <= 0, or
  * KATA_ERR_CUDA if the synchronisation or the copy failed.
  */
 KATA_API kata_status_t kata_workspace_status(const void *workspace, kata_stream_t stream);
+
+/*
+ * Self-test of the device-timeout path (failure detection without a fault).
+ * Launches one thread block that waits on an mbarrier nothing completes. The
+ * bounded wait the tensor-core kernels use gives up after 2 s of GPU time;
+ * the block then frees its tensor memory and records a device timeout in the
+ * status word, as a forward kernel does when one of its waits runs out. Once
+ * the stream has run, kata_workspace_status(workspace) returns
+ * KATA_ERR_DEVICE_TIMEOUT, and the CUDA context remains usable.
+ *   workspace   device, >= 256 bytes (a status header); the status word is
+ *               reset on `stream` before the launch.
+ * Returns KATA_OK when launched; KATA_ERR_WORKSPACE for a null or short
+ * workspace (checked on the host before anything is launched); KATA_ERR_CUDA
+ * if the reset or the launch failed. Needs an sm_100a device.
+ */
+KATA_API kata_status_t kata_selftest_device_timeout(void *workspace, size_t workspace_bytes,
+                                                    kata_stream_t stream);
 
 /*
  * Optional per-kernel device timing (CUDA events), for benchmarks. Not part

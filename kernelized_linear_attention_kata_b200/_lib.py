@@ -49,6 +49,7 @@ SIGNATURES = {
     "kata_bwd_chunked": (ctypes.c_int, [_cvp, _cvp, _cvp, _cvp, _vp, _vp, _vp, _i, _i, _i, _i,
                                         _i, _i, _i, _i, _vp, _sz, _vp]),
     "kata_workspace_status": (ctypes.c_int, [_cvp, _vp]),
+    "kata_selftest_device_timeout": (ctypes.c_int, [_vp, _sz, _vp]),
     "kata_profile_enable": (ctypes.c_int, [_i]),
     "kata_profile_count": (ctypes.c_int, []),
     "kata_profile_get": (ctypes.c_int, [_i, ctypes.POINTER(ctypes.c_char_p),

@@ -197,6 +197,15 @@ def kata_workspace_status(workspace, stream=None) -> int:
     return int(lib().kata_workspace_status(_dev(workspace, "workspace"), _stream(stream)))
 
 
+def kata_selftest_device_timeout(workspace, stream=None) -> None:
+    """Launch the device-timeout self-test into `workspace` (>= 256 bytes);
+    kata_workspace_status(workspace) then reports KATA_ERR_DEVICE_TIMEOUT."""
+    st = lib().kata_selftest_device_timeout(_dev(workspace, "workspace"),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(stream))
+    check("kata_selftest_device_timeout", st)
+
+
 def profile_enable(on: bool = True) -> None:
     """Start (and clear) or stop per-kernel CUDA-event timing inside the library."""
     check("kata_profile_enable", lib().kata_profile_enable(1 if on else 0))
@@ -261,5 +270,5 @@ __all__ = [
     "kata_fwd_chunked_sequential", "kata_fwd_quadratic", "kata_decode_step",
     "kata_workspace_status", "profile_enable", "profile_read", "fwd_chunked", "fwd_quadratic", "decode_step", "_lib",
     "bwd_chunked_workspace_bytes", "kata_bwd_chunked", "bwd_chunked", "kata_chunked_state",
-    "chunked_state",
+    "chunked_state", "kata_selftest_device_timeout",
 ]

@@ -342,6 +342,15 @@ kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
   return dispatch_shape(d_k, d_v, feature, run);
 }
 
+kata_status_t kata_selftest_device_timeout(void *workspace, size_t workspace_bytes,
+                                           kata_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!workspace || workspace_bytes < kHeaderBytes) return KATA_ERR_WORKSPACE;
+  unsigned *status = reinterpret_cast<unsigned *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
+  return selftest_wait_timeout(status, stream) == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
 kata_status_t kata_workspace_status(const void *workspace, kata_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace) return KATA_ERR_WORKSPACE;

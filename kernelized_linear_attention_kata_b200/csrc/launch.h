@@ -75,6 +75,9 @@ cudaError_t tc_chunked(const ChunkedLaunch &a);
 size_t tc_chunked_agg_floats();   // floats of one segment increment
 bool fo_tc_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t fo_tc(const ChunkedLaunch &a);
+// One block that waits on a barrier nothing completes, until the bounded
+// wait's limit; leaves kStatusDeviceTimeout in *status (selftest.cu).
+cudaError_t selftest_wait_timeout(unsigned *status, cudaStream_t stream);
 size_t fo_tc_agg_floats();        // floats of one segment increment
 
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_chunked(const ChunkedLaunch &a);

@@ -133,6 +133,13 @@ def test_state_and_from_state_host_checks(lib):
               None) == L.KATA_ERR_WORKSPACE
 
 
+def test_selftest_rejects_a_missing_or_short_workspace(lib):
+    """The device-timeout self-test checks its workspace on the host and
+    launches nothing when it is null or shorter than the status header."""
+    assert lib.kata_selftest_device_timeout(None, 0, None) == L.KATA_ERR_WORKSPACE
+    assert lib.kata_selftest_device_timeout(ctypes.c_void_p(256), 255, None) == L.KATA_ERR_WORKSPACE
+
+
 def test_empty_problems_launch_nothing(lib):
     p = ctypes.c_void_p(256)
     assert lib.kata_fwd_quadratic(p, p, p, p, 0, 4, 8, 32, 64, 1, 0, None) == L.KATA_OK
