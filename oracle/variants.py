@@ -175,6 +175,44 @@ def forward_delta(q, k, v, beta, key_feature=psd_key_feature, query_feature=psd_
     return y
 
 
+def forward_delta_chunked(q, k, v, beta, C, key_feature=psd_key_feature,
+                          query_feature=psd_query_feature, return_state=False):
+    """DeltaKATA (reading 4) in chunks of C tokens. Inside a chunk starting
+    from S'_0, every state is S'_t = S'_0 + sum_{s<=t} phi(k_s) e_s^T, where
+    e_t = beta_t ([v_t, 1] - phi~(k_t)^T S'_{t-1}) is the token's correction.
+    Substituting gives a lower-triangular system for the chunk's corrections
+    E (C x (d_v + 1)):
+        e_t + beta_t sum_{s<t} A_ts e_s = beta_t ([v_t, 1] - phi~(k_t)^T S'_0),
+    with A_ts = phi~(k_t) . phi(k_s), the weight between keys t and s. Then
+        phi~(q_t)^T S'_t = phi~(q_t)^T S'_0 + sum_{s<=t} (phi~(q_t) . phi(k_s)) e_s,
+        S'_C = S'_0 + Phi(K)^T E.
+    A library triangular solve is the step for E."""
+    beta = np.asarray(beta, dtype=np.float64)
+    if beta.shape != (q.shape[0],) or np.any(beta <= 0.0) or np.any(beta > 1.0):
+        raise ValueError("beta must be [T] with entries in (0, 1]")
+    if C < 1:
+        raise ValueError("C must be >= 1")
+    fk, fqk, fq = key_feature(k), query_feature(k), query_feature(q)
+    T, d_v = q.shape[0], v.shape[1]
+    Sa = np.zeros((fk.shape[1], d_v + 1))
+    y = np.empty((T, d_v))
+    for c0 in range(0, T, C):
+        sl = slice(c0, min(c0 + C, T))
+        n = sl.stop - sl.start
+        Phi, Psi, Fq, b = fk[sl], fqk[sl], fq[sl], beta[sl]
+        U = np.concatenate([v[sl], np.ones((n, 1))], axis=1)
+        A = np.tril(Psi @ Phi.T, -1)                       # A_ts, s < t
+        M = np.eye(n) + b[:, None] * A
+        E = np.linalg.solve(M, b[:, None] * (U - Psi @ Sa))
+        R = Fq @ Sa + np.tril(Fq @ Phi.T) @ E               # phi~(q_t)^T S'_t
+        _check_den(R[:, d_v])
+        y[sl] = R[:, :d_v] / R[:, d_v:]
+        Sa = Sa + Phi.T @ E
+    if return_state:
+        return y, Sa
+    return y
+
+
 def forward_delta_unpacked(q, k, v, beta):
     """DeltaKATA-M1 with the full d_k x d_k x (d_v + 1) state (no packing):
     M_t = M_{t-1} + beta_t (k_t k_t^T) (x) ([v_t, 1] - <k_t k_t^T, M_{t-1}>),

@@ -276,3 +276,46 @@ def test_planted_mistakes_are_caught(monkeypatch):
     vd = r.standard_normal((3, 2))
     y = V.forward_delta(kd, kd, vd, np.ones(3), query_feature=O.psd_key_feature)
     assert not np.allclose(y[2], vd[2], atol=1e-6)
+
+
+@pytest.mark.parametrize("C", [1, 5, 16, 64, 100])
+def test_delta_chunked_equals_recurrent(C):
+    """The chunked delta rule (a triangular solve per chunk for the tokens'
+    corrections) gives the recurrent rule's outputs and final state, for
+    chunk sizes that divide T, leave a ragged tail, or exceed T."""
+    r = np.random.default_rng(40 + C)
+    q, k, v = rand(70, 6, 3, seed=41)
+    beta = r.uniform(0.2, 1.0, size=70)
+    y, Sa = V.forward_delta(q, k, v, beta, return_state=True)
+    yc, Sc = V.forward_delta_chunked(q, k, v, beta, C, return_state=True)
+    assert np.allclose(yc, y, rtol=1e-11, atol=1e-12)
+    assert np.allclose(Sc, Sa, rtol=1e-11, atol=1e-12)
+
+
+def test_delta_chunked_with_other_features():
+    """Mg and first-order features through the same chunked form."""
+    r = np.random.default_rng(50)
+    q, k, v = rand(45, 8, 2, seed=51)
+    kf = lambda x: V.variant_key_feature(x, V.MG, 2)  # noqa: E731
+    qf = lambda x: V.variant_query_feature(x, V.MG, 2)  # noqa: E731
+    beta = r.uniform(0.2, 1.0, size=45)
+    assert np.allclose(V.forward_delta_chunked(q, k, v, beta, 8, kf, qf),
+                       V.forward_delta(q, k, v, beta, kf, qf), rtol=1e-11, atol=1e-12)
+    kf1 = lambda x: O.key_feature(x, O.FIRST_ORDER)  # noqa: E731
+    qf1 = lambda x: O.query_feature(x, O.FIRST_ORDER)  # noqa: E731
+    beta = r.uniform(0.1, 0.5, size=45)
+    assert np.allclose(V.forward_delta_chunked(q, k, v, beta, 8, kf1, qf1),
+                       V.forward_delta(q, k, v, beta, kf1, qf1), rtol=1e-11, atol=1e-12)
+
+
+def test_delta_chunked_planted_diagonal_is_caught(monkeypatch):
+    """Counting the token's own key in its correction (tril with the
+    diagonal) changes the result."""
+    r = np.random.default_rng(60)
+    q, k, v = rand(30, 5, 2, seed=61)
+    beta = r.uniform(0.2, 1.0, size=30)
+    real_tril = np.tril
+    monkeypatch.setattr(V.np, "tril", lambda m, k=0: real_tril(m, 0))
+    planted = V.forward_delta_chunked(q, k, v, beta, 8)
+    monkeypatch.undo()
+    assert not np.allclose(planted, V.forward_delta(q, k, v, beta), atol=1e-6)
