@@ -253,9 +253,13 @@ def run_reference(args, rank, world):
         vals.append(v)
     value = statistics.mean(vals)
     cores = blas_threads()
+    # one step is the whole workload (B x T tokens); each timed step ran a
+    # bounded sample of it, so the step time is the sample's rate applied to it
+    ms_per_step = 1000.0 * w.B * w.T / value
+    sample += "; ms_per_step applies this rate to the whole step (B x T tokens)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
