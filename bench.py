@@ -199,43 +199,104 @@ class ClockSampler:
 # CPU oracle (baseline leg and --impl reference arm)
 # ---------------------------------------------------------------------------
 
-def blas_threads():
+def host_cores():
+    """CPU cores this process may run on."""
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
         return os.cpu_count() or 1
 
 
-_ORACLE_INPUTS = {}
+_THREAD_ENV = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+
+
+def _oracle_head(job):
+    """One worker's share of the CPU baseline: the oracle's chunked forward on
+    the first `n` tokens of head (b, h), read from the inputs' .npy files.
+    Returns the seconds it took."""
+    import numpy as np
+
+    import oracle as O
+    folder, b, h, n, C, feature = job
+    q, k, v = (np.asarray(np.load(os.path.join(folder, f"{x}.npy"), mmap_mode="r")[b, h, :n],
+                          dtype=np.float64) for x in "qkv")
+    t0 = time.perf_counter()
+    O.forward_chunked(q, k, v, C, feature)
+    return time.perf_counter() - t0
+
+
+class OracleBaseline:
+    """The fp64 oracle timed on the host's cores: one process per head (spawned,
+    one BLAS thread each), each running the oracle's chunked forward on its
+    head. A round runs min(cores, B*H) heads at once on the first `n` tokens
+    of each (the causal forward of a prefix is the prefix of the forward), `n`
+    chosen so that a round takes about the budget; the rate is tokens of the
+    workload (token-heads / H) per second of wall time."""
+
+    def __init__(self, w):
+        import tempfile
+
+        import numpy as np
+
+        from kernelized_linear_attention_kata_b200 import workloads as W
+        self.w = w
+        self.cores = min(host_cores(), w.B * w.H)
+        base = "/dev/shm" if os.path.isdir("/dev/shm") else None
+        self.folder = tempfile.mkdtemp(prefix="kata_oracle_", dir=base)
+        for name, t in zip("qkv", W.make_inputs(w)):
+            # the bf16-rounded inputs, exactly, as float32
+            np.save(os.path.join(self.folder, f"{name}.npy"), t.float().numpy())
+        import multiprocessing as mp
+        saved = {k: os.environ.get(k) for k in _THREAD_ENV}
+        for k in _THREAD_ENV:
+            os.environ[k] = "1"
+        try:
+            # spawn, not fork: the parent may already hold a CUDA context
+            self.pool = mp.get_context("spawn").Pool(self.cores)
+        finally:
+            for k, val in saved.items():
+                if val is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = val
+        self.n = min(w.T, 4 * w.C)
+        self.rate_per_token = None
+
+    def round(self, budget_s):
+        """One timed round. Returns (tokens/s, seconds, description)."""
+        w = self.w
+        if self.rate_per_token is not None:
+            n = int(budget_s / self.rate_per_token) // w.C * w.C
+            self.n = max(w.C, min(w.T, n))
+        heads = [divmod(bh, w.H) for bh in range(w.B * w.H)][:self.cores]
+        jobs = [(self.folder, b, h, self.n, w.C, w.feature) for b, h in heads]
+        t0 = time.perf_counter()
+        per_head = self.pool.map(_oracle_head, jobs, chunksize=1)
+        dt = time.perf_counter() - t0
+        self.rate_per_token = max(per_head) / self.n
+        token_heads = len(heads) * self.n
+        desc = (f"oracle forward_chunked (fp64 numpy, one process and one BLAS thread per head) on "
+                f"{len(heads)} of {w.B * w.H} heads at once, first {self.n} of {w.T} tokens each, "
+                f"of {w.name}: {dt:.2f} s; tokens/s = token-heads / H / s")
+        return token_heads / w.H / dt, dt, desc
+
+    def close(self):
+        import shutil
+        self.pool.terminate()
+        self.pool.join()
+        shutil.rmtree(self.folder, ignore_errors=True)
 
 
 def oracle_sample(w, budget_s):
-    """Time the oracle's chunked form, as it stands, on whole heads of the
-    workload (full length T), head after head until `budget_s` seconds of CPU
-    work have been spent. Returns (tokens/s, description of the sample)."""
-    import oracle as O
-    from kernelized_linear_attention_kata_b200 import workloads as W
-
-    if w.name not in _ORACLE_INPUTS:
-        q, k, v = W.make_inputs(w)
-        _ORACLE_INPUTS[w.name] = (W.to_f64_numpy(q), W.to_f64_numpy(k), W.to_f64_numpy(v))
-    qn, kn, vn = _ORACLE_INPUTS[w.name]
-    token_heads = 0
-    heads = 0
-    t0 = time.perf_counter()
-    for bh in range(w.B * w.H):
-        b, h = divmod(bh, w.H)
-        O.forward_chunked(qn[b, h], kn[b, h], vn[b, h], w.C, w.feature)
-        token_heads += w.T
-        heads += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return token_heads / w.H / dt, (
-        f"oracle forward_chunked (fp64 numpy) on {heads} of {w.B * w.H} heads x {w.T} tokens of "
-        f"{w.name} in {dt:.1f} s; tokens/s = token-heads processed / H / s")
+    """The CPU baseline beside the GPU number: a calibration round, then one
+    round of about `budget_s` seconds. Returns (tokens/s, cores, description)."""
+    base = OracleBaseline(w)
+    try:
+        base.round(budget_s / 10)
+        value, _, desc = base.round(budget_s)
+        return value, base.cores, desc
+    finally:
+        base.close()
 
 
 def run_reference(args, rank, world):
@@ -244,27 +305,33 @@ def run_reference(args, rank, world):
         return 0
     w = W.WORKLOADS[args.workload]
     budget = args.ref_step_budget or max(0.5, 150.0 / (args.steps + args.warmup))
-    for _ in range(args.warmup):
-        oracle_sample(w, budget_s=budget)
-    vals = []
-    sample = ""
-    for _ in range(args.steps):
-        v, sample = oracle_sample(w, budget_s=budget)
-        vals.append(v)
+    base = OracleBaseline(w)
+    try:
+        base.round(budget / 10)                      # calibration of the sample size
+        for _ in range(args.warmup):
+            base.round(budget)
+        vals, secs = [], []
+        sample = ""
+        for _ in range(args.steps):
+            v, dt, sample = base.round(budget)
+            vals.append(v)
+            secs.append(dt)
+    finally:
+        base.close()
     value = statistics.mean(vals)
-    cores = blas_threads()
-    # one step is the whole workload (B x T tokens); each timed step ran a
-    # bounded sample of it, so the step time is the sample's rate applied to it
-    ms_per_step = 1000.0 * w.B * w.T / value
-    sample += "; ms_per_step applies this rate to the whole step (B x T tokens)"
+    ms_per_step = 1000.0 * statistics.mean(secs)
+    full_step_ms = 1000.0 * w.B * w.T / value
+    sample += (f"; a step is one such round ({ms_per_step:.0f} ms); the whole workload "
+               f"(B x T tokens) at this rate would take {full_step_ms:.0f} ms")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": base.cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "projected_full_step_ms": full_step_ms,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -503,9 +570,8 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and form == "chunked":
-        val, sample = oracle_sample(W.WORKLOADS[args.workload], budget_s=args.cpu_budget)
-        cpu = {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": sample}
+        val, cores, sample = oracle_sample(W.WORKLOADS[args.workload], budget_s=args.cpu_budget)
+        cpu = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
 
     if rank == 0:
         line = {
@@ -521,9 +587,25 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def launch_ranks(n):
+    """Re-run this command as n local ranks under torch.distributed.run
+    (127.0.0.1 rendezvous on a free port); rank 0 prints the JSON line. The
+    exit status is the launcher's."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=None,
+                    help="GPUs (ranks) on this node; without a torch.distributed launcher in "
+                         "the environment, bench.py starts that many ranks itself")
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -544,9 +626,13 @@ def main():
                     help="seconds of oracle work per reference step (default: 150 s / (K + W))")
     args = ap.parse_args()
 
+    if "WORLD_SIZE" not in os.environ and (args.gpus or 1) > 1:
+        return launch_ranks(args.gpus)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus is not None and args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
     if args.impl == "reference":
         return run_reference(args, rank, world)
     if world > 1:

@@ -88,6 +88,31 @@ typedef enum { KATA_DTYPE_F32 = 0, KATA_DTYPE_BF16 = 1 } kata_dtype_t;
 
 typedef enum { KATA_FEATURE_PSD = 0, KATA_FEATURE_FIRST_ORDER = 1 } kata_feature_t;
 
+/* Kernel family a chunked-forward request runs on. */
+typedef enum {
+    KATA_PATH_NONE = 0,             /* empty problem: nothing is launched      */
+    KATA_PATH_TENSOR_CORE_PSD = 1,  /* tcgen05/TMEM kernels, bf16 PSD,
+                                       d_k = 32, d_v = 64, C in {64, 128}     */
+    KATA_PATH_TENSOR_CORE_FIRST_ORDER = 2, /* tcgen05/TMEM kernels, bf16
+                                       first-order, d_k = d_v = 64,
+                                       C in {64, 128}                          */
+    KATA_PATH_CUDA_CORE = 3         /* fp32 FFMA kernels: the fp32 path and
+                                       every other supported shape            */
+} kata_path_t;
+
+/* How kata_fwd_chunked will run a problem (see kata_fwd_chunked_plan). */
+typedef struct {
+    kata_path_t path;   /* kernel family                                      */
+    int segments;       /* segments per (b, h) of the parallel carry (the
+                           scan across chunks): 1 = sequential carry          */
+    int segment_tokens; /* tokens per segment (a multiple of the chunk the
+                           kernels compute with); segment g starts at token
+                           g * segment_tokens                                 */
+    int chunk_tokens;   /* chunk the kernels compute with: 128 on the tensor
+                           cores for C in {64, 128} (the chunked form is exact
+                           for any C, so C only schedules the work), else C   */
+} kata_plan_t;
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 KATA_API int kata_version(void);
 
@@ -106,6 +131,23 @@ KATA_API size_t kata_state_dim(int d_k, kata_feature_t feature);
  */
 KATA_API size_t kata_fwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C,
                                         kata_dtype_t dtype, kata_feature_t feature);
+
+/*
+ * The plan kata_fwd_chunked (sequential = 0) or kata_fwd_chunked_sequential
+ * (sequential = 1) follows for this problem on the CURRENT device, with q, k,
+ * v, o (and S_out, when given) 16-byte aligned as every cudaMalloc'd buffer
+ * is: which kernel family runs and how the sequence is cut into segments
+ * for the parallel carry. Nothing is launched.
+ *   out      host pointer, written on KATA_OK.
+ * Returns KATA_ERR_UNSUPPORTED for a shape the library does not build,
+ * KATA_ERR_INVALID_ARGUMENT for a negative size or a NULL `out`, and
+ * KATA_ERR_CUDA when the device cannot be queried. A request the plan sends
+ * to the tensor cores never falls back to the CUDA cores: if the
+ * tensor-core setup fails, the call returns KATA_ERR_CUDA.
+ */
+KATA_API kata_status_t kata_fwd_chunked_plan(int B, int H, int T, int d_k, int d_v, int C,
+                                             kata_dtype_t dtype, kata_feature_t feature,
+                                             int sequential, kata_plan_t *out);
 
 /*
  * Exact O(T) chunked-state causal forward (arXiv abstract: "exact O(T)
@@ -200,7 +242,10 @@ KATA_API kata_status_t kata_chunked_state(const void *k, const void *v, int B, i
  *    kata_fwd_chunked_workspace_bytes(...) > KATA_NOALLOC_SCRATCH_BYTES.
  *  - The first call on a device looks up the array's device address for that
  *    device (cudaGetSymbolAddress with the device current); make that first
- *    call before any stream capture.
+ *    call before any stream capture. The address is kept for the life of the
+ *    process: after cudaDeviceReset (or anything else that destroys the
+ *    device's primary context) it is stale, so do not call this entry point
+ *    on that device again in the same process.
  *  - All calls share the array, which keeps the last call's contents (each
  *    call clears the status word it needs to start at zero). Calls whose work
  *    overlaps on the GPU (different streams, different host threads) race on

@@ -22,10 +22,24 @@ KATA_ERR_CUDA = 4
 KATA_ERR_NONPOSITIVE_NORMALISER = 5
 KATA_ERR_DEVICE_TIMEOUT = 6
 
+KATA_PATH_NONE = 0
+KATA_PATH_TENSOR_CORE_PSD = 1
+KATA_PATH_TENSOR_CORE_FIRST_ORDER = 2
+KATA_PATH_CUDA_CORE = 3
+PATH_NAMES = {KATA_PATH_NONE: "none", KATA_PATH_TENSOR_CORE_PSD: "tensor_core_psd",
+              KATA_PATH_TENSOR_CORE_FIRST_ORDER: "tensor_core_first_order",
+              KATA_PATH_CUDA_CORE: "cuda_core"}
+
 KATA_DTYPE_F32 = 0
 KATA_DTYPE_BF16 = 1
 KATA_FEATURE_PSD = 0
 KATA_FEATURE_FIRST_ORDER = 1
+
+class KataPlan(ctypes.Structure):
+    """kata_plan_t"""
+    _fields_ = [("path", ctypes.c_int), ("segments", ctypes.c_int),
+                ("segment_tokens", ctypes.c_int), ("chunk_tokens", ctypes.c_int)]
+
 
 # Every symbol the header declares, with (restype, argtypes).
 _vp, _cvp, _i, _sz, _fp = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
@@ -35,6 +49,8 @@ SIGNATURES = {
     "kata_status_string": (ctypes.c_char_p, [_i]),
     "kata_state_dim": (ctypes.c_size_t, [_i, _i]),
     "kata_fwd_chunked_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "kata_fwd_chunked_plan": (ctypes.c_int, [_i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                             ctypes.POINTER(KataPlan)]),
     "kata_fwd_chunked": (ctypes.c_int, _FWD),
     "kata_fwd_chunked_sequential": (ctypes.c_int, _FWD),
     "kata_fwd_chunked_noalloc": (ctypes.c_int, [_cvp, _cvp, _cvp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,

@@ -64,6 +64,18 @@ def chunked_workspace_bytes(B, H, T, d_k, d_v, C, dtype=torch.bfloat16, feature=
                                                       _feature(feature)))
 
 
+def fwd_chunked_plan(B, H, T, d_k, d_v, C, dtype=torch.bfloat16, feature="psd",
+                     sequential=False) -> dict:
+    """How kata_fwd_chunked runs this problem on the current device (16-byte
+    aligned buffers): {"path", "segments", "segment_tokens", "chunk_tokens"}."""
+    p = _lib.KataPlan()
+    check("kata_fwd_chunked_plan",
+          lib().kata_fwd_chunked_plan(B, H, T, d_k, d_v, C, _DTYPES[dtype], _feature(feature),
+                                      1 if sequential else 0, ctypes.byref(p)))
+    return {"path": _lib.PATH_NAMES.get(p.path, str(p.path)), "segments": p.segments,
+            "segment_tokens": p.segment_tokens, "chunk_tokens": p.chunk_tokens}
+
+
 def alloc_workspace(B, H, T, d_k, d_v, C, dtype=torch.bfloat16, feature="psd", device=None):
     n = chunked_workspace_bytes(B, H, T, d_k, d_v, C, dtype, feature)
     if n == 0:
@@ -270,5 +282,5 @@ __all__ = [
     "kata_fwd_chunked_sequential", "kata_fwd_quadratic", "kata_decode_step",
     "kata_workspace_status", "profile_enable", "profile_read", "fwd_chunked", "fwd_quadratic", "decode_step", "_lib",
     "bwd_chunked_workspace_bytes", "kata_bwd_chunked", "bwd_chunked", "kata_chunked_state",
-    "chunked_state", "kata_selftest_device_timeout",
+    "chunked_state", "kata_selftest_device_timeout", "fwd_chunked_plan",
 ]

@@ -61,7 +61,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     procs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, *ARCH_FLAGS, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-dc" if False else "-c",
+        cmd = [nvcc, *ARCH_FLAGS, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c",
                src, "-o", obj, *(extra or [])]
         if verbose:
             print(" ".join(cmd), flush=True)

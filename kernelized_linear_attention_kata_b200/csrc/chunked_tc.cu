@@ -920,12 +920,8 @@ size_t tc_chunked_agg_floats() { return (size_t)kAggFloats; }
 cudaError_t tc_chunked(const ChunkedLaunch &a) {
   // segments of whole 128-token chunks, no more of them than the caller
   // sized the workspace for
-  const int nchunks = (a.T + kC - 1) / kC;
-  int G = a.G < 1 ? 1 : a.G;
-  if (G > nchunks) G = nchunks;
-  const int per = (nchunks + G - 1) / G;
-  G = (nchunks + per - 1) / per;
-  const int seg_len = per * kC;
+  int G, seg_len;
+  tile_segments(a.T, kC, a.G, &G, &seg_len);
   // the state-only call reads neither q nor o: their maps are built on k, v
   // and never used by the increment kernel
   CUtensorMap tq, tk, tv, to;
@@ -933,7 +929,7 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
       !make_tma_3d_bf16(&tk, a.k, kDK, a.T, a.BH, kC) ||
       !make_tma_3d_bf16(&tv, a.v, kDV, a.T, a.BH, kC) ||
       !make_tma_3d_bf16(&to, a.state_only ? a.v : a.o, kDV, a.T, a.BH, kC))
-    return cudaErrorNotSupported;
+    return cudaErrorInvalidValue;              // accepted shape: a failure, not a fallback
   cudaError_t e;
   // increments of segments 0 .. G-2 (all G for the state-only call)
   const int G_inc = a.state_only ? G : G - 1;

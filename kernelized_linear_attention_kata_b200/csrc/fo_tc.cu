@@ -516,12 +516,8 @@ bool fo_tc_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int featur
 cudaError_t fo_tc(const ChunkedLaunch &a) {
   // segments of whole 128-token tiles, no more of them than the caller sized
   // the workspace for
-  const int ntiles = (a.T + kTile - 1) / kTile;
-  int G = a.G < 1 ? 1 : a.G;
-  if (G > ntiles) G = ntiles;
-  const int per = (ntiles + G - 1) / G;
-  G = (ntiles + per - 1) / per;
-  const int seg_len = per * kTile;
+  int G, seg_len;
+  tile_segments(a.T, kTile, a.G, &G, &seg_len);
   // the state-only call reads neither q nor o: their maps are built on k, v
   // and never used by the increment kernel
   CUtensorMap tq, tk, tv, to;
@@ -529,7 +525,7 @@ cudaError_t fo_tc(const ChunkedLaunch &a) {
       !make_tma_3d_bf16(&tk, a.k, kDh, a.T, a.BH, kTile) ||
       !make_tma_3d_bf16(&tv, a.v, kDh, a.T, a.BH, kTile) ||
       !make_tma_3d_bf16(&to, a.state_only ? a.v : a.o, kDh, a.T, a.BH, kTile))
-    return cudaErrorNotSupported;
+    return cudaErrorInvalidValue;              // accepted shape: a failure, not a fallback
   cudaError_t e;
   // increments of segments 0 .. G-2 (all G for the state-only call)
   const int G_inc = a.state_only ? G : G - 1;

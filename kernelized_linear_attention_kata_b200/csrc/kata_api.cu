@@ -108,16 +108,31 @@ kata_status_t dispatch_shape(int d_k, int d_v, kata_feature_t feature, F &&f) {
   return KATA_ERR_UNSUPPORTED;
 }
 
+// Kernel family of a chunked request: decided from the shape and the
+// pointers' alignment only, so that kata_fwd_chunked_plan reports exactly
+// what a call runs.
+kata_path_t chunked_path(const ChunkedLaunch &a, int d_k, int d_v, int C, kata_dtype_t dtype,
+                         int feature) {
+  if (a.BH == 0 || a.T == 0) return KATA_PATH_NONE;
+  if (dtype == KATA_DTYPE_BF16 && tc_chunked_supported(a, d_k, d_v, C, feature))
+    return KATA_PATH_TENSOR_CORE_PSD;
+  if (dtype == KATA_DTYPE_BF16 && fo_tc_supported(a, d_k, d_v, C, feature))
+    return KATA_PATH_TENSOR_CORE_FIRST_ORDER;
+  return KATA_PATH_CUDA_CORE;
+}
+
 struct ChunkedRun {
   kata_dtype_t dtype;
   ChunkedLaunch a;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
-    cudaError_t e = cudaErrorNotSupported;
-    if (dtype == KATA_DTYPE_BF16 && tc_chunked_supported(a, DK, DV, a.C, FEAT)) e = tc_chunked(a);
-    else if (dtype == KATA_DTYPE_BF16 && fo_tc_supported(a, DK, DV, a.C, FEAT)) e = fo_tc(a);
-    if (e == cudaErrorNotSupported)
-      e = dtype == KATA_DTYPE_F32 ? simt_chunked<DK, DV, FEAT, float>(a)
-                                  : simt_chunked<DK, DV, FEAT, __nv_bfloat16>(a);
+    cudaError_t e;
+    switch (chunked_path(a, DK, DV, a.C, dtype, FEAT)) {
+      case KATA_PATH_TENSOR_CORE_PSD: e = tc_chunked(a); break;
+      case KATA_PATH_TENSOR_CORE_FIRST_ORDER: e = fo_tc(a); break;
+      default:
+        e = dtype == KATA_DTYPE_F32 ? simt_chunked<DK, DV, FEAT, float>(a)
+                                    : simt_chunked<DK, DV, FEAT, __nv_bfloat16>(a);
+    }
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
   }
 };
@@ -223,6 +238,33 @@ size_t kata_state_dim(int d_k, kata_feature_t feature) {
   if (feature == KATA_FEATURE_PSD) return (size_t)d_k * (d_k + 1) / 2;
   if (feature == KATA_FEATURE_FIRST_ORDER) return (size_t)d_k + 1;
   return 0;
+}
+
+kata_status_t kata_fwd_chunked_plan(int B, int H, int T, int d_k, int d_v, int C,
+                                    kata_dtype_t dtype, kata_feature_t feature, int sequential,
+                                    kata_plan_t *out) {
+  if (B < 0 || H < 0 || T < 0 || C <= 0 || !out) return KATA_ERR_INVALID_ARGUMENT;
+  if (!supported(d_k, d_v, C, dtype, feature)) return KATA_ERR_UNSUPPORTED;
+  const int sms = device_sm_count();
+  if (sms <= 0) return KATA_ERR_CUDA;
+  const long long BH = (long long)B * H;
+  const Split sp = segment_split(BH, T, C, sms, sequential != 0);
+  // 16-byte aligned stand-ins for the caller's buffers (never dereferenced)
+  void *aligned = reinterpret_cast<void *>(uintptr_t(256));
+  ChunkedLaunch a{aligned, aligned, aligned, aligned, BH, T, C, nullptr, nullptr, nullptr,
+                  nullptr, sp.G, sp.seg_len, nullptr};
+  kata_plan_t p{};
+  p.path = chunked_path(a, d_k, d_v, C, dtype, feature);
+  if (p.path == KATA_PATH_TENSOR_CORE_PSD || p.path == KATA_PATH_TENSOR_CORE_FIRST_ORDER) {
+    p.chunk_tokens = 128;
+    tile_segments(T, 128, sp.G, &p.segments, &p.segment_tokens);
+  } else {
+    p.chunk_tokens = C;
+    p.segments = sp.G;
+    p.segment_tokens = sp.seg_len;
+  }
+  *out = p;
+  return KATA_OK;
 }
 
 size_t kata_fwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C,

@@ -51,8 +51,13 @@ extern "C" kata_status_t kata_fwd_chunked_noalloc(const void *q, const void *k, 
                                                   kata_feature_t feature, float *S_out,
                                                   float *z_out, kata_stream_t stream) {
   if (B < 0 || H < 0 || T < 0 || C <= 0) return KATA_ERR_INVALID_ARGUMENT;
+  // the plan query tells an unsupported shape (KATA_ERR_UNSUPPORTED) from a
+  // device that cannot be queried (KATA_ERR_CUDA)
+  kata_plan_t plan;
+  const kata_status_t pst = kata_fwd_chunked_plan(B, H, T, d_k, d_v, C, dtype, feature, 0, &plan);
+  if (pst != KATA_OK) return pst;
   const size_t need = kata_fwd_chunked_workspace_bytes(B, H, T, d_k, d_v, C, dtype, feature);
-  if (need == 0) return KATA_ERR_UNSUPPORTED;
+  if (need == 0) return KATA_ERR_CUDA;
   if (need > (size_t)KATA_NOALLOC_SCRATCH_BYTES) return KATA_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KATA_ERR_CUDA;

@@ -66,9 +66,23 @@ struct BackwardLaunch {
   cudaStream_t stream;
 };
 
-// Tensor-core kernels (bf16 only). They return cudaErrorNotSupported, having
-// launched nothing, for shapes or alignments they do not handle; the caller
-// then runs the CUDA-core kernel instead.
+// Segments of whole `tile`-token tiles for the tensor-core kernels, no more
+// of them than the caller sized the workspace for (G_req).
+inline void tile_segments(int T, int tile, int G_req, int *G, int *seg_len) {
+  const int ntiles = (T + tile - 1) / tile;
+  int g = G_req < 1 ? 1 : G_req;
+  if (g > ntiles) g = ntiles;
+  if (g < 1) g = 1;
+  const int per = (ntiles + g - 1) / g;
+  *G = per > 0 ? (ntiles + per - 1) / per : 1;
+  *seg_len = per * tile;
+}
+
+// Tensor-core kernels (bf16 only). The chunked kernels' *_supported
+// predicates decide, from the shape and the pointers' alignment alone,
+// whether a request runs on them; tc_quadratic returns cudaErrorNotSupported,
+// having launched nothing, for the shapes it does not take. Once a kernel
+// has accepted a request it either launches or fails: no fallback.
 cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature);
 bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t tc_chunked(const ChunkedLaunch &a);

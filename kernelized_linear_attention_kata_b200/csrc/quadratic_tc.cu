@@ -273,7 +273,7 @@ cudaError_t launch(const QuadraticLaunch &a) {
   if (!make_tma_3d_bf16(&tq, a.q, DK, a.T, a.BH, kBlock) ||
       !make_tma_3d_bf16(&tk, a.k, DK, a.T, a.BH, kBlock) ||
       !make_tma_3d_bf16(&tv, a.v, kDV, a.T, a.BH, kBlock))
-    return cudaErrorNotSupported;
+    return cudaErrorInvalidValue;              // accepted shape: a failure, not a fallback
   // 1 KB alignment slack; at least 100 KB so that at most two CTAs (two
   // 256-column TMEM allocations) share an SM.
   const int smem = L::kBytes + 1024 < 100 * 1024 ? 100 * 1024 : L::kBytes + 1024;
@@ -290,8 +290,9 @@ cudaError_t launch(const QuadraticLaunch &a) {
 }  // namespace
 
 // Tensor-core quadratic forward for bf16, d_v = 64, d_k in {16, 32, 64}.
-// Returns cudaErrorNotSupported when the shape or alignment is not handled
-// here (the caller then uses the CUDA-core kernel).
+// Returns cudaErrorNotSupported, having launched nothing, when the shape or
+// alignment is not handled here (the caller then uses the CUDA-core kernel);
+// for a shape it accepts it either launches or returns an error.
 cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature) {
   if (d_v != kDV || a.BH > 65535 || a.T <= 0) return cudaErrorNotSupported;
   for (const void *p : {a.q, a.k, a.v, (const void *)a.o})

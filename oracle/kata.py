@@ -89,7 +89,7 @@ def psd_key_feature(x: np.ndarray) -> np.ndarray:
     """Packed psi(x) = x x^T, upper triangle: [..., d_k] -> [..., D]."""
     d_k = x.shape[-1]
     iu, ju = np.triu_indices(d_k)          # same order as psd_pairs
-    return x[..., iu] * x[..., ju]
+    return np.take(x, iu, axis=-1) * np.take(x, ju, axis=-1)
 
 
 def psd_query_feature(x: np.ndarray) -> np.ndarray:
@@ -101,7 +101,7 @@ def psd_query_feature(x: np.ndarray) -> np.ndarray:
     d_k = x.shape[-1]
     iu, ju = np.triu_indices(d_k)
     mult = np.where(iu == ju, 1.0, 2.0)
-    return x[..., iu] * x[..., ju] * mult
+    return np.take(x, iu, axis=-1) * np.take(x, ju, axis=-1) * mult
 
 
 def first_order_feature(x: np.ndarray) -> np.ndarray:

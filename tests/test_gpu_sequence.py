@@ -7,9 +7,9 @@ sequence-sharded forward would: each slice's state from kata_chunked_state,
 the carry into slice r = the sum of the states of slices 0 .. r-1, each
 slice's outputs from kata_fwd_chunked_from_state. The concatenated outputs
 must match the definition on the whole sequence (per-row bound of the
-forward: 1e-4 fp32, 2e-2 bf16), and the last slice's final state the whole
-sequence's (1e-4 of the largest entry; 1e-2 for the bf16 PSD tensor-core
-path, whose update multiplies bf16-rounded key products).
+forward: 1e-4 fp32, 2e-2 bf16), and the states the oracle's element by
+element, within the bounds of each kernel family's arithmetic
+(tests/state_bounds.py).
 """
 
 import numpy as np
@@ -20,6 +20,7 @@ import oracle as O
 from kernelized_linear_attention_kata_b200 import api
 from kernelized_linear_attention_kata_b200 import build as kbuild
 from kernelized_linear_attention_kata_b200 import workloads as W
+from state_bounds import assert_state_close, tc_psd_path
 
 pytestmark = pytest.mark.gpu
 
@@ -36,23 +37,6 @@ def cuda_lib():
 def rel_rows(y, ref):
     y = np.asarray(y, dtype=np.float64)
     return float(np.max(np.max(np.abs(y - ref), -1) / np.maximum(np.max(np.abs(ref), -1), 1e-6)))
-
-
-def oracle_state(k, v, feature):
-    kn, vn = f64(k), f64(v)
-    B, H = kn.shape[:2]
-    D = O.state_dim(kn.shape[3], feature)
-    S = np.empty((B, H, D, vn.shape[3]))
-    z = np.empty((B, H, D))
-    for b in range(B):
-        for h in range(H):
-            S[b, h], z[b, h] = O.final_state(kn[b, h], vn[b, h], feature)
-    return S, z
-
-
-def state_tol(dtype, feature, d_k, d_v, C):
-    tc_psd = dtype == "bf16" and feature == "psd" and (d_k, d_v) == (32, 64) and C in (64, 128)
-    return 1e-2 if tc_psd else 1e-4
 
 
 # (feature, dtype, B, H, T, d_k, d_v, C, slice boundaries): the tensor-core
@@ -75,10 +59,8 @@ def test_state_only_matches_oracle(case):
                    seed=500 + T, recipe="unit")
     q, k, v = W.make_inputs(w)
     S, z = api.chunked_state(k.cuda(), v.cuda(), C, feature)
-    S_ref, z_ref = oracle_state(k, v, feature)
-    tol = state_tol(dtype, feature, d_k, d_v, C)
-    assert np.max(np.abs(S.cpu().numpy() - S_ref)) <= tol * np.max(np.abs(S_ref))
-    assert np.max(np.abs(z.cpu().numpy() - z_ref)) <= tol * np.max(np.abs(z_ref))
+    assert_state_close(S.cpu().numpy(), z.cpu().numpy(), f64(k), f64(v), feature,
+                       tc_psd_path(dtype, feature, d_k, d_v, C), "state only")
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c[:8])))
@@ -103,17 +85,20 @@ def test_slices_from_carried_state_match_whole_sequence(case):
         # it: the previous carry plus this slice's own state
         Sl, zl = api.chunked_state(ks, vs, C, feature)
         S0, z0 = S0 + Sl, z0 + zl
-        # the forward's own final state agrees with that carry
-        tol_s = state_tol(dtype, feature, d_k, d_v, C)
-        assert torch.max(torch.abs(S_out - S0)) <= tol_s * torch.max(torch.abs(S0))
+        # the forward's own final state and that carry are both the state of
+        # tokens 0 .. b - 1 (the carry is a sum of up to len(cuts) - 1
+        # separately rounded slice states)
+        kb, vb = f64(k[:, :, :b]), f64(v[:, :, :b])
+        tc = tc_psd_path(dtype, feature, d_k, d_v, C)
+        assert_state_close(S_out.cpu().numpy(), z_out.cpu().numpy(), kb, vb, feature, tc,
+                           f"forward's state after token {b}", scale=float(len(cuts)))
+        assert_state_close(S0.cpu().numpy(), z0.cpu().numpy(), kb, vb, feature, tc,
+                           f"carry after token {b}", scale=float(len(cuts)))
     y = torch.cat(outs, dim=2).float().cpu().numpy()
     ref = O.per_head(O.forward_brute_force, f64(q), f64(k), f64(v), feature)
     tol = 1e-4 if dtype == "f32" else 2e-2
     assert rel_rows(y, ref) <= tol
-    S_ref, z_ref = oracle_state(k, v, feature)
-    tol_s = state_tol(dtype, feature, d_k, d_v, C)
-    assert np.max(np.abs(S0.cpu().numpy() - S_ref)) <= tol_s * np.max(np.abs(S_ref))
-    assert np.max(np.abs(z0.cpu().numpy() - z_ref)) <= tol_s * np.max(np.abs(z_ref))
+
 
 
 def test_from_state_with_no_tokens_returns_the_state():

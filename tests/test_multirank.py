@@ -187,3 +187,36 @@ def test_sequence_sharded_forward_equals_the_whole_sequence(world, feature):
         S_ref, z_ref = O.final_state(k[0, h], v[0, h], feature)
         assert np.allclose(res[world - 1][1][0, h], S_ref, rtol=1e-12, atol=1e-12)
         assert np.allclose(res[world - 1][2][0, h], z_ref, rtol=1e-12, atol=1e-12)
+
+
+def _bench_lines(argv, env=None):
+    import json
+    import subprocess
+    e = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        e.pop(k, None)
+    e.update(env or {})
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *argv], env=e,
+                       capture_output=True, text=True, timeout=300)
+    lines = [json.loads(l) for l in p.stdout.splitlines() if l.startswith("{")]
+    return p.returncode, lines, p.stderr
+
+
+def test_bench_starts_its_own_ranks():
+    """`bench.py --gpus 2` without a launcher in the environment re-runs itself
+    as two ranks under torch.distributed.run; rank 0 alone prints the line,
+    with n_gpus = 2 (reference arm: the CPU oracle, so no GPU is needed)."""
+    rc, lines, err = _bench_lines(["--gpus", "2", "--impl", "reference", "--steps", "1",
+                                   "--warmup", "0", "--workload", "tiny_f32",
+                                   "--ref-step-budget", "0.2"])
+    assert rc == 0, err[-2000:]
+    assert len(lines) == 1, lines
+    assert lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_bench_rejects_a_rank_count_the_launcher_did_not_start():
+    rc, lines, err = _bench_lines(["--gpus", "3", "--impl", "reference", "--steps", "1",
+                                   "--warmup", "0", "--workload", "tiny_f32"],
+                                  env={"WORLD_SIZE": "2", "RANK": "0", "LOCAL_RANK": "0"})
+    assert rc != 0 and not lines
+    assert "--gpus 3" in err
