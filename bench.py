@@ -102,8 +102,9 @@ def load_peaks():
 # Source files that define each profiled kernel (a recorded traffic figure is
 # valid only while these are unchanged).
 KERNEL_SOURCES = {
-    "tc_segment_pass": ["chunked_tc.cu", "tc_common.cuh", "common.cuh"],
-    "tc_segment_increment": ["chunked_tc.cu", "tc_common.cuh", "common.cuh"],
+    "tc_segment_pass": ["psd_pair_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
+    "tc_segment_increment": ["psd_increment_tc.cu", "psd_tc_common.cuh", "tc_common.cuh",
+                             "common.cuh"],
     "tc_quadratic": ["quadratic_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_fo_pass": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_fo_increment": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],

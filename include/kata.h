@@ -32,6 +32,11 @@
  *                    of the off-diagonal pairs on the query side).
  *      FIRST_ORDER : D = d_k + 1, row 0 is the constant feature 1, row 1 + i
  *                    is k_i; weight 1 + <q_t, k_s>.
+ *      MULTI_PSD2  : D = 2 h (h + 1) / 2 with h = d_k / 2: the packed rows
+ *                    (i <= j, row-major) of slice 1, then those of slice 2;
+ *                    S[r] = sum_s k_si k_sj v_s with (i, j) in one slice.
+ *      SUMMED_PSD2 : D = h (h + 1) / 2, row r <-> (i, j), i <= j < h;
+ *                    S[r] = sum_s (k_si k_sj + k_s(h+i) k_s(h+j)) v_s.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream). Argument errors are detected on the host and returned
  *    before anything is launched. KATA_ERR_CUDA reports a launch error
@@ -50,6 +55,8 @@
  * Supported shapes (anything else returns KATA_ERR_UNSUPPORTED):
  *    PSD          d_k in {16, 32}
  *    FIRST_ORDER  d_k in {16, 32, 64}
+ *    MULTI_PSD2, SUMMED_PSD2  d_k in {16, 32} (forward forms and the decode
+ *                 step; kata_bwd_chunked takes PSD and FIRST_ORDER only)
  *    d_v in {16, 32, 64};  C in {16, 32, 64, 128};  T >= 0;
  *    T need not be a multiple of C (the last chunk is shorter).
  */
@@ -86,7 +93,22 @@ typedef enum {
 
 typedef enum { KATA_DTYPE_F32 = 0, KATA_DTYPE_BF16 = 1 } kata_dtype_t;
 
-typedef enum { KATA_FEATURE_PSD = 0, KATA_FEATURE_FIRST_ORDER = 1 } kata_feature_t;
+/*
+ * Feature maps. The two-factor variants are the KATA-Mg and KATA-Sigma-g of
+ * the explainer (section 2.3, g = 2), which names them without a
+ * construction; the library reads the factors of a head vector x in R^d_k
+ * as its two halves x_1, x_2 in R^(d_k / 2):
+ *   KATA_FEATURE_MULTI_PSD2   phi(x) = [x_1 x_1^T, x_2 x_2^T] (KATA-Mg, g = 2),
+ *                             weight <q_1,k_1>^2 + <q_2,k_2>^2;
+ *   KATA_FEATURE_SUMMED_PSD2  Psi(x) = x_1 x_1^T + x_2 x_2^T (KATA-Sigma-g,
+ *                             g = 2), weight sum_{a,b} <q_a,k_b>^2.
+ */
+typedef enum {
+    KATA_FEATURE_PSD = 0,
+    KATA_FEATURE_FIRST_ORDER = 1,
+    KATA_FEATURE_MULTI_PSD2 = 2,
+    KATA_FEATURE_SUMMED_PSD2 = 3
+} kata_feature_t;
 
 /* Kernel family a chunked-forward request runs on. */
 typedef enum {

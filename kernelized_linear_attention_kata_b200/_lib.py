@@ -34,6 +34,8 @@ KATA_DTYPE_F32 = 0
 KATA_DTYPE_BF16 = 1
 KATA_FEATURE_PSD = 0
 KATA_FEATURE_FIRST_ORDER = 1
+KATA_FEATURE_MULTI_PSD2 = 2      # KATA-Mg, g = 2
+KATA_FEATURE_SUMMED_PSD2 = 3     # KATA-Sigma-g, g = 2
 
 class KataPlan(ctypes.Structure):
     """kata_plan_t"""

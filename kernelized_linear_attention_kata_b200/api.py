@@ -18,7 +18,8 @@ from ._lib import (KATA_DTYPE_BF16, KATA_DTYPE_F32, KATA_FEATURE_FIRST_ORDER, KA
                    check, lib)
 
 _DTYPES = {torch.float32: KATA_DTYPE_F32, torch.bfloat16: KATA_DTYPE_BF16}
-_FEATURES = {"psd": KATA_FEATURE_PSD, "first_order": KATA_FEATURE_FIRST_ORDER}
+_FEATURES = {"psd": KATA_FEATURE_PSD, "first_order": KATA_FEATURE_FIRST_ORDER,
+             "mg2": _lib.KATA_FEATURE_MULTI_PSD2, "sigma_g2": _lib.KATA_FEATURE_SUMMED_PSD2}
 
 
 def _feature(feature: str) -> int:

@@ -22,6 +22,8 @@ bool supported(int d_k, int d_v, int C, kata_dtype_t dtype, kata_feature_t featu
     if (d_k != 16 && d_k != 32) return false;
   } else if (feature == KATA_FEATURE_FIRST_ORDER) {
     if (d_k != 16 && d_k != 32 && d_k != 64) return false;
+  } else if (feature == KATA_FEATURE_MULTI_PSD2 || feature == KATA_FEATURE_SUMMED_PSD2) {
+    if (d_k != 16 && d_k != 32) return false;
   } else {
     return false;
   }
@@ -64,8 +66,20 @@ size_t increment_floats(int D, int d_k, int d_v) {
   return simt > tc ? simt : tc;
 }
 
-size_t workspace_bytes_for(long long BH, int D, int d_k, int d_v, const Split &sp) {
-  const size_t agg = (size_t)BH * (size_t)sp.G * increment_floats(D, d_k, d_v) * sizeof(float);
+// Increments per head a chunked request keeps in its workspace: one per
+// segment, or, on the PSD tensor-core path, one per piece of a segment.
+size_t increments_per_head(kata_path_t path, long long BH, int T, int sms, bool sequential,
+                           const Split &sp) {
+  if (path == KATA_PATH_TENSOR_CORE_PSD && !sequential) {   // the sequential carry needs none
+    int G, seg_len, P;
+    tc_chunked_layout(BH, T, sms, sequential, &G, &seg_len, &P);
+    return (size_t)G * (size_t)P;
+  }
+  return (size_t)sp.G;
+}
+
+size_t workspace_bytes_for(long long BH, int D, int d_k, int d_v, size_t incs_per_head) {
+  const size_t agg = (size_t)BH * incs_per_head * increment_floats(D, d_k, d_v) * sizeof(float);
   return kHeaderBytes + align_up(agg, kAlign);
 }
 
@@ -88,7 +102,7 @@ BwdLayout bwd_layout(long long BH, int T, int D, int d_v, const Split &sp) {
 
 // Calls F::template run<DK, DV, FEAT>() for the runtime (d_k, d_v, feature).
 template <typename F>
-kata_status_t dispatch_shape(int d_k, int d_v, kata_feature_t feature, F &&f) {
+kata_status_t dispatch_shape(int d_k, int d_v, kata_feature_t feature, F &f) {
 #define KATA_DV_CASES(DK, FEAT)                                         \
   switch (d_v) {                                                        \
     case 16: return f.template operator()<DK, 16, FEAT>();              \
@@ -99,10 +113,18 @@ kata_status_t dispatch_shape(int d_k, int d_v, kata_feature_t feature, F &&f) {
   if (feature == KATA_FEATURE_PSD) {
     if (d_k == 16) { KATA_DV_CASES(16, kPSD) }
     if (d_k == 32) { KATA_DV_CASES(32, kPSD) }
-  } else {
+  } else if (feature == KATA_FEATURE_FIRST_ORDER) {
     if (d_k == 16) { KATA_DV_CASES(16, kFirstOrder) }
     if (d_k == 32) { KATA_DV_CASES(32, kFirstOrder) }
     if (d_k == 64) { KATA_DV_CASES(64, kFirstOrder) }
+  } else if constexpr (!F::kBaseFeaturesOnly) {
+    if (feature == KATA_FEATURE_MULTI_PSD2) {
+      if (d_k == 16) { KATA_DV_CASES(16, kMg2) }
+      if (d_k == 32) { KATA_DV_CASES(32, kMg2) }
+    } else if (feature == KATA_FEATURE_SUMMED_PSD2) {
+      if (d_k == 16) { KATA_DV_CASES(16, kSg2) }
+      if (d_k == 32) { KATA_DV_CASES(32, kSg2) }
+    }
   }
 #undef KATA_DV_CASES
   return KATA_ERR_UNSUPPORTED;
@@ -122,6 +144,7 @@ kata_path_t chunked_path(const ChunkedLaunch &a, int d_k, int d_v, int C, kata_d
 }
 
 struct ChunkedRun {
+  static constexpr bool kBaseFeaturesOnly = false;
   kata_dtype_t dtype;
   ChunkedLaunch a;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
@@ -138,6 +161,7 @@ struct ChunkedRun {
 };
 
 struct QuadraticRun {
+  static constexpr bool kBaseFeaturesOnly = false;
   kata_dtype_t dtype;
   QuadraticLaunch a;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
@@ -151,6 +175,7 @@ struct QuadraticRun {
 };
 
 struct BackwardRun {
+  static constexpr bool kBaseFeaturesOnly = true;     // the gradient covers PSD and first-order
   kata_dtype_t dtype;
   BackwardLaunch a;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
@@ -161,6 +186,7 @@ struct BackwardRun {
 };
 
 struct DecodeRun {
+  static constexpr bool kBaseFeaturesOnly = false;
   kata_dtype_t dtype;
   DecodeLaunch a;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
@@ -186,8 +212,18 @@ kata_status_t chunked_common(const void *q, const void *k, const void *v, void *
   const int sms = device_sm_count();
   if (sms <= 0) return KATA_ERR_CUDA;
   const Split sp = segment_split(BH, T, C, sms, sequential);
-  if (workspace_bytes < workspace_bytes_for(BH, D, d_k, d_v, sp)) return KATA_ERR_WORKSPACE;
   unsigned char *ws = static_cast<unsigned char *>(workspace);
+  ChunkedLaunch a{q, k, v, o, BH, T, C, S_out, z_out, reinterpret_cast<unsigned *>(ws),
+                  reinterpret_cast<float *>(ws + kHeaderBytes), sp.G, sp.seg_len, stream};
+  a.S0 = S0;
+  a.z0 = z0;
+  a.state_only = state_only;
+  a.sms = sms;
+  a.sequential = sequential;
+  const kata_path_t path = chunked_path(a, d_k, d_v, C, dtype, feature);
+  if (workspace_bytes <
+      workspace_bytes_for(BH, D, d_k, d_v, increments_per_head(path, BH, T, sms, sequential, sp)))
+    return KATA_ERR_WORKSPACE;
   if (BH == 0 || T == 0) {
     // no tokens: the state out is the initial state (zero if none is given)
     if (cudaMemsetAsync(ws, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
@@ -203,13 +239,7 @@ kata_status_t chunked_common(const void *q, const void *k, const void *v, void *
     return KATA_OK;
   }
   if (!k || !v || (!state_only && (!q || !o))) return KATA_ERR_INVALID_ARGUMENT;
-  unsigned *status = reinterpret_cast<unsigned *>(ws);
-  if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
-  ChunkedLaunch a{q, k, v, o, BH, T, C, S_out, z_out, status,
-                  reinterpret_cast<float *>(ws + kHeaderBytes), sp.G, sp.seg_len, stream};
-  a.S0 = S0;
-  a.z0 = z0;
-  a.state_only = state_only;
+  if (cudaMemsetAsync(a.status, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
   ChunkedRun run{dtype, a};
   return dispatch_shape(d_k, d_v, feature, run);
 }
@@ -237,6 +267,10 @@ size_t kata_state_dim(int d_k, kata_feature_t feature) {
   if (d_k <= 0) return 0;
   if (feature == KATA_FEATURE_PSD) return (size_t)d_k * (d_k + 1) / 2;
   if (feature == KATA_FEATURE_FIRST_ORDER) return (size_t)d_k + 1;
+  if (d_k % 2) return 0;
+  const size_t h = (size_t)d_k / 2;
+  if (feature == KATA_FEATURE_MULTI_PSD2) return h * (h + 1);
+  if (feature == KATA_FEATURE_SUMMED_PSD2) return h * (h + 1) / 2;
   return 0;
 }
 
@@ -255,7 +289,11 @@ kata_status_t kata_fwd_chunked_plan(int B, int H, int T, int d_k, int d_v, int C
                   nullptr, sp.G, sp.seg_len, nullptr};
   kata_plan_t p{};
   p.path = chunked_path(a, d_k, d_v, C, dtype, feature);
-  if (p.path == KATA_PATH_TENSOR_CORE_PSD || p.path == KATA_PATH_TENSOR_CORE_FIRST_ORDER) {
+  if (p.path == KATA_PATH_TENSOR_CORE_PSD) {
+    int P;
+    p.chunk_tokens = 128;
+    tc_chunked_layout(BH, T, sms, sequential != 0, &p.segments, &p.segment_tokens, &P);
+  } else if (p.path == KATA_PATH_TENSOR_CORE_FIRST_ORDER) {
     p.chunk_tokens = 128;
     tile_segments(T, 128, sp.G, &p.segments, &p.segment_tokens);
   } else {
@@ -275,7 +313,14 @@ size_t kata_fwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, i
   if (sms <= 0) return 0;
   const long long BH = (long long)B * H;
   const Split sp = segment_split(BH, T, C, sms, false);
-  return workspace_bytes_for(BH, (int)kata_state_dim(d_k, feature), d_k, d_v, sp);
+  // the forward needs at least what the sequential carry needs, so one size
+  // serves both entry points; the path is the one 16-byte aligned buffers take
+  void *aligned = reinterpret_cast<void *>(uintptr_t(256));
+  ChunkedLaunch a{aligned, aligned, aligned, aligned, BH, T, C, nullptr, nullptr, nullptr,
+                  nullptr, sp.G, sp.seg_len, nullptr};
+  const kata_path_t path = chunked_path(a, d_k, d_v, C, dtype, feature);
+  return workspace_bytes_for(BH, (int)kata_state_dim(d_k, feature), d_k, d_v,
+                             increments_per_head(path, BH, T, sms, false, sp));
 }
 
 kata_status_t kata_fwd_chunked(const void *q, const void *k, const void *v, void *o, int B, int H,
@@ -345,6 +390,7 @@ kata_status_t kata_decode_step(const void *q, const void *k, const void *v, floa
 size_t kata_bwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, int C,
                                         kata_dtype_t dtype, kata_feature_t feature) {
   if (B < 0 || H < 0 || T < 0 || C <= 0) return 0;
+  if (feature != KATA_FEATURE_PSD && feature != KATA_FEATURE_FIRST_ORDER) return 0;
   if (!supported(d_k, d_v, C, dtype, feature)) return 0;
   const int sms = device_sm_count();
   if (sms <= 0) return 0;
@@ -361,6 +407,7 @@ kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (B < 0 || H < 0 || T < 0 || C <= 0) return KATA_ERR_INVALID_ARGUMENT;
   if (!supported(d_k, d_v, C, dtype, feature)) return KATA_ERR_UNSUPPORTED;
+  if (feature != KATA_FEATURE_PSD && feature != KATA_FEATURE_FIRST_ORDER) return KATA_ERR_UNSUPPORTED;
   if (!workspace) return KATA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return KATA_ERR_WORKSPACE;
   const int sms = device_sm_count();

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace kata {
@@ -23,6 +24,8 @@ struct ChunkedLaunch {
   const float *S0 = nullptr, *z0 = nullptr;
   // only the state after the T tokens (S_out, z_out); q and o are not read
   bool state_only = false;
+  int sms = 0;             // SMs of the device (the tensor-core kernels size their grids by it)
+  bool sequential = false; // one segment per head (the sequential carry)
 };
 
 // Sum of the G segment increments of each head, written as the state in the
@@ -87,6 +90,16 @@ cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature
 bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t tc_chunked(const ChunkedLaunch &a);
 size_t tc_chunked_agg_floats();   // floats of one segment increment
+// The PSD tensor-core forward's split: G segments of seg_len tokens per head,
+// each segment's increment computed as P pieces (G * P increments per head in
+// the workspace).
+void tc_chunked_layout(long long BH, int T, int sms, bool sequential, int *G, int *seg_len, int *P);
+// Increments of segments 0 .. G_inc - 1 (cps chunks each), P pieces per
+// segment, into agg[bh][g P + j] ([528 x 64] + [32 x 32] fp32 each, the PSD
+// tensor-core layout), incs_per_head increments per head in agg.
+cudaError_t psd_tc_increments(const CUtensorMap &tk, const CUtensorMap &tv, float *agg,
+                              unsigned *status, long long BH, int T, int G_inc, int P, int cps,
+                              int incs_per_head, cudaStream_t stream);
 bool fo_tc_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t fo_tc(const ChunkedLaunch &a);
 // One block that waits on a barrier nothing completes, until the bounded

@@ -131,10 +131,12 @@ __device__ __forceinline__ void fill_row_table(int4 *tab, int tid, int nthreads)
 }
 
 // phi_q(q)_r for a row-table entry, q read from shared memory.
-template <int FEAT>
+template <int DK, int FEAT>
 __device__ __forceinline__ float query_feature_row(const float *qt, int4 e) {
-  if constexpr (FEAT == kPSD) {
+  if constexpr (FEAT == kPSD || FEAT == kMg2) {
     return __int_as_float(e.z) * qt[e.x] * qt[e.y];
+  } else if constexpr (FEAT == kSg2) {
+    return __int_as_float(e.z) * fmaf(qt[e.x], qt[e.y], qt[DK / 2 + e.x] * qt[DK / 2 + e.y]);
   } else {
     return e.x < 0 ? 1.f : qt[e.x];
   }
@@ -208,7 +210,7 @@ segment_pass_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
       // inter-chunk readout phi_q(q_t)^T S_c, phi_q(q_t)^T z_c
 #pragma unroll 4
       for (int r = 0; r < D; ++r) {
-        const float ph = query_feature_row<FEAT>(qt, tab[r]);
+        const float ph = query_feature_row<DK, FEAT>(qt, tab[r]);
         const float4 *sr = reinterpret_cast<const float4 *>(S + r * DV + vb * VB);
 #pragma unroll
         for (int c4 = 0; c4 < VB / 4; ++c4) {
@@ -223,13 +225,10 @@ segment_pass_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
       float qv[DK];
 #pragma unroll
       for (int i = 0; i < DK; ++i) qv[i] = qt[i];
-      // intra-chunk block: weights (q_t . k_s)^2 (or 1 + q_t . k_s), s <= t
+      // intra-chunk block: the weights of the keys s <= t (closed form)
       for (int s = 0; s <= t; ++s) {
         const float *kr = ks + s * DK;
-        float dot = 0.f;
-#pragma unroll
-        for (int i = 0; i < DK; ++i) dot = fmaf(qv[i], kr[i], dot);
-        const float w = FEAT == kPSD ? dot * dot : 1.f + dot;
+        const float w = pair_weight<DK, FEAT>(qv, kr);
         den += w;
         const float4 *vr = reinterpret_cast<const float4 *>(vs + s * DV + vb * VB);
 #pragma unroll
@@ -327,10 +326,7 @@ __global__ void quadratic_kernel(const Tin *__restrict__ q, const Tin *__restric
     const int smax = min(n, t - s0 + 1);   // keys s0 .. t within this block
     for (int s = 0; s < smax; ++s) {
       const float *kr = ks + s * DK;
-      float dot = 0.f;
-#pragma unroll
-      for (int i = 0; i < DK; ++i) dot = fmaf(qv[i], kr[i], dot);
-      const float w = FEAT == kPSD ? dot * dot : 1.f + dot;
+      const float w = pair_weight<DK, FEAT>(qv, kr);
       den += w;
       const float4 *vr = reinterpret_cast<const float4 *>(vs + s * DV + vb * VB);
 #pragma unroll

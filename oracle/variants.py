@@ -131,6 +131,18 @@ def forward_variant_brute_force(q, k, v, variant, g):
     return (W @ v) / den[:, None]
 
 
+def forward_variant_rows(q, k, v, rows, variant, g):
+    """Rows `rows` of the causal output from the definition, each in O(t):
+    the closed-form weights of keys 0..t for query t [LA definition]."""
+    out = np.empty((len(rows), v.shape[1]))
+    for n, t in enumerate(rows):
+        w = variant_weights(q[t:t + 1], k[:t + 1], variant, g)[0]
+        den = w.sum()
+        _check_den(np.array([den]))
+        out[n] = (w @ v[:t + 1]) / den
+    return out
+
+
 def forward_variant_recurrent(q, k, v, variant, g, return_state=False):
     """The same output from the packed state: S_t = S_{t-1} + phi(k_t) v_t^T,
     z_t = z_{t-1} + phi(k_t), y_t = phi~(q_t)^T S_t / phi~(q_t)^T z_t."""

@@ -363,8 +363,10 @@ def test_unsupported_shape_raises():
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("B,H,T", [(1, 1, 1), (1, 2, 127), (1, 3, 128), (2, 2, 129), (1, 4, 1000),
-                                   (1, 2, 5000), (2, 80, 300)])
+                                   (1, 2, 5000), (2, 80, 300), (1, 1, 150 * 128 + 5)])
 def test_tc_chunked_c128_shapes_and_state(B, H, T):
+    """Tensor-core PSD path against the oracle, outputs and state. The last
+    shape has segments of two chunks whose increments are cut into pieces."""
     w = W.Workload("tc", B=B, H=H, T=T, d_k=32, d_v=64, C=128, dtype="bf16", feature="psd",
                    seed=1000 + T + H, recipe="unit")
     q, k, v = W.make_inputs(w)

@@ -75,6 +75,16 @@ def test_recurrent_equals_brute_force(variant, g):
     assert np.allclose(a, b, rtol=1e-11, atol=1e-12)
 
 
+@pytest.mark.parametrize("variant,g", [(V.MG, 2), (V.SIGMA_G, 2)])
+def test_rows_form_equals_brute_force(variant, g):
+    """The per-row form (used on long sequences) is the brute force's rows."""
+    q, k, v = rand(70, 8, 5, seed=13)
+    rows = np.array([0, 1, 2, 33, 68, 69])
+    a = V.forward_variant_brute_force(q, k, v, variant, g)[rows]
+    b = V.forward_variant_rows(q, k, v, rows, variant, g)
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
 def test_state_dims_order_m1_above_m2():
     """Reading 1 gives M1 the largest state at a fixed d_k [JA 5]: 528 rows at
     d_k = 32, 272 for M2 (two 16-wide factors), 136 for Sigma-2."""
