@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+from dataclasses import replace
 import json
 import os
 import statistics
@@ -46,29 +47,58 @@ KERNEL_BOUND = {
     "simt_bwd_dkdv": "alu",
     "simt_bwd_prefix_increment": "alu",
     "simt_bwd_suffix_increment": "alu",
+    "simt_delta": "alu",
 }
 METRIC_BWD = "KATA causal bwd (dq, dk, dv) tokens/sec at T=131072 (chunked)"
 
 
+def state_rows(d_k, feature):
+    """D, the state rows of a feature (PSD, first-order, KATA-Mg / Sigma-g
+    with g = 2 over the two halves of the key)."""
+    h = d_k // 2
+    return {"psd": d_k * (d_k + 1) // 2, "first_order": d_k + 1, "mg2": h * (h + 1),
+            "sigma_g2": h * (h + 1) // 2}[feature]
+
+
+def pair_weight_flops(d_k, feature):
+    """Flops of one query-key weight in closed form: the dot product(s) and
+    their squares (PSD (q.k)^2; first-order 1 + q.k; Mg2 two half-dots;
+    Sigma-g2 four half-dots)."""
+    return {"psd": 2 * d_k + 1, "first_order": 2 * d_k + 1, "mg2": 2 * d_k + 3,
+            "sigma_g2": 4 * d_k + 7}[feature]
+
+
 def algorithmic_per_token_head(d_k, d_v, C, feature="psd"):
     """(flops, bytes) the chunked forward must do per token-head: the causal
-    half of the intra-chunk block, the state update and the readout; bf16
-    q, k, v read once and o written once."""
-    D = d_k * (d_k + 1) // 2 if feature == "psd" else d_k + 1
-    intra = (C + 1) / 2 * (2 * d_k + 2 * d_v + 2)
+    half of the intra-chunk block (each pair: its weight, the d_v
+    multiply-adds of the value and the normaliser's add), the state update
+    and the readout; bf16 q, k, v read once and o written once."""
+    D = state_rows(d_k, feature)
+    intra = (C + 1) / 2 * (pair_weight_flops(d_k, feature) + 2 * d_v + 1)
     update = 2 * D * d_v + D
     readout = 2 * D * d_v + 2 * D
     return intra + update + readout, (2 * d_k + d_v) * 2 + d_v * 2
 
 
+def algorithmic_delta_per_token_head(d_k, d_v):
+    """(flops, bytes) of the DeltaKATA rule per token-head, as the recurrence
+    states it: the stored binding phi~(k)^T S', the rank-one write and the
+    readout phi~(q)^T S', each over the D x (d_v + 1) augmented state; bf16
+    q, k, v and fp32 beta read once, o written once."""
+    D = state_rows(d_k, "psd")
+    return 6 * D * (d_v + 1), (2 * d_k + d_v) * 2 + 4 + d_v * 2
+
+
 def feature_products_per_token_head(d_k, feature="psd"):
     """Scalar products the feature expansion needs per token-head: phi(k) for
     the state update and phi~(q) for the readout, one product per packed
-    feature each (the query's multiplicity 2 folds into its product). The
-    first-order feature [1, u] is the input itself and needs none."""
-    if feature != "psd":
+    feature each (the query's multiplicity 2 folds into its product; a
+    Sigma-g2 feature sums two). The first-order feature [1, u] is the input
+    itself and needs none."""
+    if feature == "first_order":
         return 0
-    return 2 * (d_k * (d_k + 1) // 2)
+    per = 2 if feature == "sigma_g2" else 1
+    return 2 * per * state_rows(d_k, feature)
 
 
 def algorithmic_backward_per_token_head(d_k, d_v, C, feature="psd"):
@@ -102,9 +132,8 @@ def load_peaks():
 # Source files that define each profiled kernel (a recorded traffic figure is
 # valid only while these are unchanged).
 KERNEL_SOURCES = {
-    "tc_segment_pass": ["psd_pair_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
-    "tc_segment_increment": ["psd_increment_tc.cu", "psd_tc_common.cuh", "tc_common.cuh",
-                             "common.cuh"],
+    "tc_segment_pass": ["chunked_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
+    "tc_segment_increment": ["chunked_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
     "tc_quadratic": ["quadratic_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_fo_pass": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_fo_increment": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
@@ -379,12 +408,16 @@ def run_ours(args, rank, world, local_rank):
     kbuild.build()
     dev = torch.device("cuda", local_rank)
     form = args.form
-    w = W.WORKLOADS[args.workload if form != "first_order" else "first_order64k_bf16"]
+    fo = form in ("first_order", "first_order_sequential")
+    w = W.WORKLOADS[args.workload if not fo else "first_order64k_bf16"]
+    if args.feature:
+        if fo or form in ("backward", "delta"):
+            raise SystemExit("--feature applies to the chunked, sequential, quadratic forms")
+        w = replace(w, feature=args.feature)
     if form == "quadratic":
         w = w.with_T(args.T or W.LONG_QUADRATIC_T)
     elif args.T:
         w = w.with_T(args.T)
-    from dataclasses import replace
     seq = args.shard == "sequence"
     if seq and (form != "chunked" or w.T % world):
         raise SystemExit("--shard sequence needs --form chunked and T divisible by the ranks")
@@ -426,6 +459,14 @@ def run_ours(args, rank, world, local_rank):
                 api.kata_bwd_chunked(q, k, v, dy, dq, dk, dv, w.C, w.feature, workspace=ws)
             flops_th, bytes_th = algorithmic_backward_per_token_head(w.d_k, w.d_v, w.C, w.feature)
             e2e_in, e2e_out = [q, k, v, dy], [dq, dk, dv]
+        elif form == "delta":
+            beta = W.make_delta_beta(w.B, w.H, w.T, w.seed, device=dev)
+            ws = torch.empty(256, dtype=torch.uint8, device=dev)
+
+            def step():
+                api.kata_fwd_delta(q, k, v, beta, o, w.feature, workspace=ws)
+            flops_th, bytes_th = algorithmic_delta_per_token_head(w.d_k, w.d_v)
+            phi_th = 3 * state_rows(w.d_k, "psd")
         elif form == "quadratic":
             ws = None
 
@@ -449,7 +490,7 @@ def run_ours(args, rank, world, local_rank):
             phi_th = feature_products_per_token_head(w.d_k, w.feature)
         else:
             ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
-            seq_carry = form == "sequential"
+            seq_carry = form in ("sequential", "first_order_sequential")
 
             def step():
                 api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws, sequential=seq_carry)
@@ -461,7 +502,9 @@ def run_ours(args, rank, world, local_rank):
         config["form"] = {"chunked": "chunked (segmented scan carry)",
                           "sequential": "chunked (sequential carry)",
                           "first_order": "chunked first-order (segmented scan carry)",
+                          "first_order_sequential": "chunked first-order (sequential carry)",
                           "quadratic": "quadratic (flash-style)",
+                          "delta": "DeltaKATA (delta-rule state, chunked triangular solve)",
                           "backward": "gradient of the chunked form (prefix and suffix scans)"}[form]
 
     def barrier():
@@ -612,12 +655,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long131k_bf16")
     ap.add_argument("--form", default="chunked",
-                    choices=["chunked", "sequential", "first_order", "quadratic", "decode", "backward"],
+                    choices=["chunked", "sequential", "first_order", "first_order_sequential",
+                             "quadratic", "decode", "backward", "delta"],
                     help="chunked is the headline; the others are secondary measurements")
     ap.add_argument("--shard", choices=["heads", "sequence"], default="heads",
                     help="heads: independent replicas, one batch per rank (weak scaling); "
                          "sequence: one sequence cut along T, one slice per rank, one all-reduce "
                          "of the slice states (strong scaling)")
+    ap.add_argument("--feature", choices=["psd", "mg2", "sigma_g2"], default=None,
+                    help="feature map of the chunked / sequential / quadratic forms (default: the "
+                         "workload's, PSD); mg2 and sigma_g2 are KATA-Mg and KATA-Sigma-g, g = 2")
     ap.add_argument("--decode-batch", type=int, default=W_DECODE_BATCH)
     ap.add_argument("--T", type=int, default=0, help="override T (profiling a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")

@@ -356,9 +356,45 @@ KATA_API kata_status_t kata_bwd_chunked(const void *q, const void *k, const void
                                         kata_stream_t stream);
 
 /*
+ * DeltaKATA forward: the delta-rule state update that the KATA explainer
+ * (section 4, "DeltaKATA") credits with correcting stale bindings at
+ * repeated keys. The pages give no rule; the library reads it as the delta
+ * rule on the state augmented with its normaliser, S' = [S | z] (D rows,
+ * d_v + 1 columns), with a per-token write strength beta_t in (0, 1]:
+ *   S'_t = S'_(t-1) + beta_t phi(k_t) ([v_t, 1] - phi_q(k_t)^T S'_(t-1)),
+ *   y_t  = (phi_q(q_t)^T S'_t)[:d_v] / (phi_q(q_t)^T S'_t)[d_v]
+ * (phi the key-side, phi_q the query-side packed PSD feature; the current
+ * token's write is read, as in the additive forward). For a unit key
+ * phi_q(k) . phi(k) = |k|^4 = 1, so beta = 1 overwrites the binding stored
+ * at a repeated key; keys orthogonal in feature space give the additive
+ * state with weights beta. Computed in chunks of 32 tokens (an exact form:
+ * a triangular solve per chunk), one thread block per (b, h), fp32 on the
+ * CUDA cores for both element types.
+ *   q, k, v, o         as kata_fwd_chunked.
+ *   beta               device fp32 [B, H, T], entries in (0, 1] (not
+ *                      checked on the device; other values give the rule's
+ *                      arithmetic without its meaning).
+ *   S0                 optional device fp32 [B, H, D, d_v + 1]: the state
+ *                      before the first token (library PSD row order, the
+ *                      normaliser in column d_v); NULL is zero.
+ *   S_out              optional device fp32 [B, H, D, d_v + 1]: the state
+ *                      after the last token.
+ *   workspace          device, >= 256 bytes, 256-byte aligned: the status
+ *                      word (kata_workspace_status reports a non-positive
+ *                      normaliser as for the forward).
+ * Feature: PSD with d_k in {16, 32}, d_v in {16, 32, 64}; anything else
+ * returns KATA_ERR_UNSUPPORTED.
+ */
+KATA_API kata_status_t kata_fwd_delta(const void *q, const void *k, const void *v,
+                                      const float *beta, void *o, int B, int H, int T, int d_k,
+                                      int d_v, kata_dtype_t dtype, kata_feature_t feature,
+                                      const float *S0, float *S_out, void *workspace,
+                                      size_t workspace_bytes, kata_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the status word a kata_fwd_chunked(...),
  * kata_fwd_chunked_sequential(...), kata_fwd_chunked_from_state(...),
- * kata_chunked_state(...), kata_bwd_chunked(...) or
+ * kata_chunked_state(...), kata_bwd_chunked(...), kata_fwd_delta(...) or
  * kata_selftest_device_timeout(...) call left in `workspace`: KATA_OK, or
  * KATA_ERR_DEVICE_TIMEOUT if a bounded wait inside a kernel gave up (the
  * kernel returned early, its outputs are undefined, the context is usable),

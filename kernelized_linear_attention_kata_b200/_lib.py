@@ -66,6 +66,8 @@ SIGNATURES = {
     "kata_bwd_chunked_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i, _i]),
     "kata_bwd_chunked": (ctypes.c_int, [_cvp, _cvp, _cvp, _cvp, _vp, _vp, _vp, _i, _i, _i, _i,
                                         _i, _i, _i, _i, _vp, _sz, _vp]),
+    "kata_fwd_delta": (ctypes.c_int, [_cvp, _cvp, _cvp, _fp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                      _fp, _fp, _vp, _sz, _vp]),
     "kata_workspace_status": (ctypes.c_int, [_cvp, _vp]),
     "kata_selftest_device_timeout": (ctypes.c_int, [_vp, _sz, _vp]),
     "kata_profile_enable": (ctypes.c_int, [_i]),

@@ -205,6 +205,40 @@ def kata_bwd_chunked(q, k, v, dout, dq, dk, dv, C, feature="psd", workspace=None
     return dq, dk, dv
 
 
+def kata_fwd_delta(q, k, v, beta, o, feature="psd", S0=None, S_out=None, workspace=None,
+                   stream=None):
+    """DeltaKATA forward into `o` (see include/kata.h): beta [B, H, T] fp32
+    write strengths; S0 / S_out optional [B, H, D, d_v + 1] fp32 states."""
+    B, H, T, d_k, d_v = _shapes(q, k, v, o)
+    if tuple(beta.shape) != (B, H, T):
+        raise ValueError("beta must be [B, H, T] fp32")
+    D = state_dim(d_k, feature)
+    for t, name in ((S0, "S0"), (S_out, "S_out")):
+        if t is not None and tuple(t.shape) != (B, H, D, d_v + 1):
+            raise ValueError(f"{name} must be [B, H, {D}, {d_v + 1}] fp32")
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=q.device)
+    st = lib().kata_fwd_delta(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+                              _dev(beta, "beta", torch.float32), _dev(o, "o"), B, H, T, d_k, d_v,
+                              _dtype(q), _feature(feature), _opt(S0, "S0"), _opt(S_out, "S_out"),
+                              _dev(workspace, "workspace"),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    check("kata_fwd_delta", st)
+    return o
+
+
+def fwd_delta(q, k, v, beta, feature="psd", return_state=False, S0=None):
+    """(o) or (o, S') of the DeltaKATA forward, allocated with torch."""
+    o = torch.empty_like(v)
+    S = None
+    if return_state:
+        B, H, _, d_k = q.shape
+        S = torch.empty((B, H, state_dim(d_k, feature), v.shape[3] + 1), dtype=torch.float32,
+                        device=q.device)
+    kata_fwd_delta(q, k, v, beta, o, feature, S0=S0, S_out=S)
+    return (o, S) if return_state else o
+
+
 def kata_workspace_status(workspace, stream=None) -> int:
     """Synchronises the stream and returns the status code left in the workspace."""
     return int(lib().kata_workspace_status(_dev(workspace, "workspace"), _stream(stream)))
@@ -283,5 +317,6 @@ __all__ = [
     "kata_fwd_chunked_sequential", "kata_fwd_quadratic", "kata_decode_step",
     "kata_workspace_status", "profile_enable", "profile_read", "fwd_chunked", "fwd_quadratic", "decode_step", "_lib",
     "bwd_chunked_workspace_bytes", "kata_bwd_chunked", "bwd_chunked", "kata_chunked_state",
-    "chunked_state", "kata_selftest_device_timeout", "fwd_chunked_plan",
+    "chunked_state", "kata_selftest_device_timeout", "fwd_chunked_plan", "kata_fwd_delta",
+    "fwd_delta",
 ]

@@ -431,6 +431,42 @@ kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
   return dispatch_shape(d_k, d_v, feature, run);
 }
 
+kata_status_t kata_fwd_delta(const void *q, const void *k, const void *v, const float *beta,
+                             void *o, int B, int H, int T, int d_k, int d_v, kata_dtype_t dtype,
+                             kata_feature_t feature, const float *S0, float *S_out,
+                             void *workspace, size_t workspace_bytes, kata_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (B < 0 || H < 0 || T < 0) return KATA_ERR_INVALID_ARGUMENT;
+  if (feature != KATA_FEATURE_PSD || !supported(d_k, d_v, 0, dtype, feature)) return KATA_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < kHeaderBytes) return KATA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0) return KATA_ERR_WORKSPACE;
+  const long long BH = (long long)B * H;
+  if (BH > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
+  unsigned *status = reinterpret_cast<unsigned *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
+  const int D = (int)kata_state_dim(d_k, feature);
+  if (BH == 0 || T == 0) {
+    const size_t sb = (size_t)BH * D * (d_v + 1) * sizeof(float);
+    if (S_out && BH > 0 &&
+        (S0 ? cudaMemcpyAsync(S_out, S0, sb, cudaMemcpyDeviceToDevice, stream)
+            : cudaMemsetAsync(S_out, 0, sb, stream)) != cudaSuccess)
+      return KATA_ERR_CUDA;
+    return KATA_OK;
+  }
+  if (!q || !k || !v || !beta || !o) return KATA_ERR_INVALID_ARGUMENT;
+  const DeltaLaunch a{q, k, v, beta, o, S0, S_out, status, BH, T, stream};
+  cudaError_t e = cudaErrorNotSupported;
+#define KATA_DELTA_CASE(DK, DV)                                                      \
+  if (d_k == DK && d_v == DV)                                                        \
+    e = dtype == KATA_DTYPE_F32 ? simt_delta<DK, DV, float>(a)                       \
+                                : simt_delta<DK, DV, __nv_bfloat16>(a);
+  KATA_DELTA_CASE(16, 16) KATA_DELTA_CASE(16, 32) KATA_DELTA_CASE(16, 64)
+  KATA_DELTA_CASE(32, 16) KATA_DELTA_CASE(32, 32) KATA_DELTA_CASE(32, 64)
+#undef KATA_DELTA_CASE
+  if (e == cudaErrorNotSupported) return KATA_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
 kata_status_t kata_selftest_device_timeout(void *workspace, size_t workspace_bytes,
                                            kata_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);

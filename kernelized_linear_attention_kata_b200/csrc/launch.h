@@ -46,6 +46,22 @@ struct QuadraticLaunch {
   cudaStream_t stream;
 };
 
+// DeltaKATA forward (simt_delta.cu): q, k, v, o as the chunked forward; beta
+// [BH][T] fp32 write strengths; S0 / S_out nullable [BH][D][d_v + 1] fp32
+// (the state augmented with its normaliser column, library row order).
+struct DeltaLaunch {
+  const void *q, *k, *v;
+  const float *beta;
+  void *o;
+  const float *S0;
+  float *S_out;
+  unsigned *status;
+  long long BH;
+  int T;
+  cudaStream_t stream;
+};
+template <int DK, int DV, typename Tin> cudaError_t simt_delta(const DeltaLaunch &a);
+
 struct DecodeLaunch {
   const void *q, *k, *v;
   float *S, *z;
@@ -94,12 +110,7 @@ size_t tc_chunked_agg_floats();   // floats of one segment increment
 // each segment's increment computed as P pieces (G * P increments per head in
 // the workspace).
 void tc_chunked_layout(long long BH, int T, int sms, bool sequential, int *G, int *seg_len, int *P);
-// Increments of segments 0 .. G_inc - 1 (cps chunks each), P pieces per
-// segment, into agg[bh][g P + j] ([528 x 64] + [32 x 32] fp32 each, the PSD
-// tensor-core layout), incs_per_head increments per head in agg.
-cudaError_t psd_tc_increments(const CUtensorMap &tk, const CUtensorMap &tv, float *agg,
-                              unsigned *status, long long BH, int T, int G_inc, int P, int cps,
-                              int incs_per_head, cudaStream_t stream);
+
 bool fo_tc_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t fo_tc(const ChunkedLaunch &a);
 // One block that waits on a barrier nothing completes, until the bounded

@@ -161,64 +161,5 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 __device__ __forceinline__ void warp_arrive(uint64_t *bar) { tc::mbar_arrive(bar); }
 
 
-// Key features in tensor memory (the A operand of a TS update MMA: lane =
-// feature, columns = tokens, two bf16 per column). The key-side warps first
-// transpose the chunk's K tile into K^T [32 dims][128 tokens] in shared
-// memory (rows padded to 272 bytes, so that 32 threads reading 16 bytes of
-// 32 different rows hit every bank group four times, the minimum); thread l
-// then holds row l of K^T in registers and takes a partner row from another
-// lane of its warp by shuffles. A tile is written and consumed in two
-// halves of 64 tokens (32 columns), so that two 32-column buffers already
-// let the production of one half overlap the MMAs of the other.
-constexpr int kKtPitch = 272;
-constexpr int kKtBytes = 32 * kKtPitch;
-
-// This thread's token `token` of the K tile (64-byte rows, 64-byte swizzle)
-// into column `token` of K^T.
-__device__ __forceinline__ void transpose_k(const uint8_t *ktile, uint8_t *kt, int token) {
-  uint32_t x[16];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(ktile + sw64(token, c));
-    x[4 * c + 0] = v.x;
-    x[4 * c + 1] = v.y;
-    x[4 * c + 2] = v.z;
-    x[4 * c + 3] = v.w;
-  }
-#pragma unroll
-  for (int d = 0; d < 32; ++d)
-    *reinterpret_cast<uint16_t *>(kt + d * kKtPitch + 2 * token) =
-        (uint16_t)(x[d >> 1] >> (16 * (d & 1)));
-}
-
-// Row `row` of K^T (dimension `row` of the chunk's 128 tokens, two tokens
-// per word) into registers.
-__device__ __forceinline__ void load_kt_row(const uint8_t *kt, int row, uint32_t (&X)[64]) {
-  const uint4 *a = reinterpret_cast<const uint4 *>(kt + row * kKtPitch);
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint4 x = a[c];
-    X[4 * c + 0] = x.x;
-    X[4 * c + 1] = x.y;
-    X[4 * c + 2] = x.z;
-    X[4 * c + 3] = x.w;
-  }
-}
-
-// Half H (tokens 64 H .. 64 H + 63) of the tile row of feature (l, src): the
-// products of this thread's dimension (X) with lane src's, taken by a warp
-// shuffle, into 32 tensor-memory columns (one bf16 rounding per product);
-// `zero` writes zeros (lanes that carry no feature).
-template <int H>
-__device__ __forceinline__ void key_half(uint32_t taddr, const uint32_t (&X)[64], int src, bool zero) {
-  uint32_t w[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    const uint32_t y = __shfl_sync(0xffffffffu, X[32 * H + c], src);
-    w[c] = zero ? 0u : bmul2(X[32 * H + c], y);
-  }
-  tc::tmem_st32(taddr, w);
-}
-
 }  // namespace psd
 }  // namespace kata

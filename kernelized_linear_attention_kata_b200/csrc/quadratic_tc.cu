@@ -300,12 +300,12 @@ cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature
   if (feature == kPSD) {
     if (d_k == 16) return launch<16, kPSD>(a);
     if (d_k == 32) return launch<32, kPSD>(a);
-  } else {
+  } else if (feature == kFirstOrder) {
     if (d_k == 16) return launch<16, kFirstOrder>(a);
     if (d_k == 32) return launch<32, kFirstOrder>(a);
     if (d_k == 64) return launch<64, kFirstOrder>(a);
   }
-  return cudaErrorNotSupported;
+  return cudaErrorNotSupported;                  // other features: the CUDA-core kernel
 }
 
 }  // namespace kata

@@ -157,3 +157,13 @@ def make_decode_prior_tokens(batch, heads, n_tokens=DECODE_PRIOR_TOKENS, d_k=DEC
 def to_f64_numpy(t: torch.Tensor):
     """Exact widening of the rounded inputs for the oracle."""
     return t.detach().to("cpu", torch.float64).numpy()
+
+
+def make_delta_beta(B, H, T, seed, device="cpu"):
+    """DeltaKATA write strengths [B, H, T] fp32: uniform in (0, 1], with
+    every fourth token at exactly 1 (a full overwrite)."""
+    g = _generator(seed + 313, device)
+    u = torch.rand((B, H, T), generator=g, device=device, dtype=torch.float32)
+    beta = 1.0 - u * 0.9                      # (0.1, 1]
+    beta[..., ::4] = 1.0
+    return beta.contiguous()

@@ -78,11 +78,41 @@ def test_host_rejects_unsupported_shapes(lib):
     assert _fwd(lib, d_v=48) == L.KATA_ERR_UNSUPPORTED
     assert _fwd(lib, C=96) == L.KATA_ERR_UNSUPPORTED
     assert _fwd(lib, dtype=5) == L.KATA_ERR_UNSUPPORTED
-    assert _fwd(lib, feature=3) == L.KATA_ERR_UNSUPPORTED
+    assert _fwd(lib, feature=7) == L.KATA_ERR_UNSUPPORTED
+    # the two-factor variants need an even d_k the library builds (16 or 32)
+    assert _fwd(lib, feature=L.KATA_FEATURE_MULTI_PSD2, d_k=64) == L.KATA_ERR_UNSUPPORTED
+    assert _fwd(lib, feature=L.KATA_FEATURE_SUMMED_PSD2, d_k=24) == L.KATA_ERR_UNSUPPORTED
     assert _fwd(lib, fn="kata_fwd_chunked_sequential", d_k=8) == L.KATA_ERR_UNSUPPORTED
     p = ctypes.c_void_p(256)
     assert lib.kata_fwd_quadratic(p, p, p, p, 1, 1, 8, 24, 64, 1, 0, None) == L.KATA_ERR_UNSUPPORTED
     assert lib.kata_decode_step(p, p, p, p, p, p, 1, 1, 32, 40, 1, 0, None) == L.KATA_ERR_UNSUPPORTED
+
+
+def test_variant_state_dims(lib):
+    assert lib.kata_state_dim(32, L.KATA_FEATURE_MULTI_PSD2) == 2 * 136
+    assert lib.kata_state_dim(32, L.KATA_FEATURE_SUMMED_PSD2) == 136
+    assert lib.kata_state_dim(16, L.KATA_FEATURE_MULTI_PSD2) == 2 * 36
+    assert lib.kata_state_dim(15, L.KATA_FEATURE_SUMMED_PSD2) == 0
+
+
+def test_delta_host_checks(lib):
+    p = ctypes.c_void_p(256)
+
+    def delta(feature=L.KATA_FEATURE_PSD, d_k=32, d_v=64, B=1, ws=p, ws_bytes=256):
+        return lib.kata_fwd_delta(p, p, p, p, p, B, 1, 16, d_k, d_v, L.KATA_DTYPE_BF16, feature,
+                                  None, None, ws, ws_bytes, None)
+    assert delta(feature=L.KATA_FEATURE_FIRST_ORDER) == L.KATA_ERR_UNSUPPORTED
+    assert delta(feature=L.KATA_FEATURE_MULTI_PSD2) == L.KATA_ERR_UNSUPPORTED
+    assert delta(d_k=24) == L.KATA_ERR_UNSUPPORTED
+    assert delta(B=-1) == L.KATA_ERR_INVALID_ARGUMENT
+    assert delta(ws=ctypes.c_void_p(0)) == L.KATA_ERR_WORKSPACE
+    assert delta(ws_bytes=100) == L.KATA_ERR_WORKSPACE
+    assert delta(ws=ctypes.c_void_p(256 + 16)) == L.KATA_ERR_WORKSPACE
+
+
+def test_backward_rejects_the_variants(lib):
+    assert lib.kata_bwd_chunked_workspace_bytes(1, 1, 16, 32, 64, 64, L.KATA_DTYPE_BF16,
+                                                L.KATA_FEATURE_MULTI_PSD2) == 0
 
 
 def test_host_rejects_bad_arguments(lib):
