@@ -1,0 +1,579 @@
+// Tensor-core (tcgen05 / TMEM / TMA) gradient of the chunked PSD forward,
+// bf16 inputs, d_k = 32, d_v = 64, fp32 accumulation.
+//
+// The chain rule of y_t = sum_(s<=t) w_ts v_s / sum_(s<=t) w_ts with
+// w_ts = (q_t . k_s)^2 (KATA explainer section 2.3: the exact chunked form;
+// arXiv abstract: the models are trained with these kernels): with
+// d_t = sum_(s<=t) w_ts, n_t = sum_(s<=t) w_ts v_s, g_t = dout_t / d_t and
+// c_t = -(dout_t . n_t) / d_t^2,
+//   e_ts = g_t . v_s + c_t                       (dL/dw_ts, s <= t)
+//   dq_t = sum_(s<=t) e_ts 2 (q_t . k_s) k_s.
+// Inside a chunk of 128 tokens this is a dense block; the earlier chunks
+// enter through the prefix state (S, Z) of the forward:
+//   dout_t . n_t (carried) = phi_q(q_t) . (S dout_t),  d_t (carried) = q_t^T Z q_t,
+//   dq_t (carried)         = J(q_t)^T (S dout_t) / d_t + 2 c_t Z q_t,
+// J the Jacobian of the query feature. Per chunk (bf16 operands, fp32
+// accumulators in tensor memory):
+//   A  = Q K^T, D' = dout V^T                  the intra-chunk blocks, in two
+//                                              halves of 64 keys
+//   X  = dout S^T                              64 features at a time; the
+//                                              CUDA cores contract X with the
+//                                              query features and their
+//                                              Jacobian
+//   U  = Q Z
+//   M  = 2 A (D' / d_t + c_t), masked to s <= t, then dq += M K
+//   S += phi(K)^T V,  Z += K^T K               the forward's update.
+// The kernel writes dq and, per token, d_t and c_t for the suffix pass.
+//
+// Parallel carry: the forward's segment increments (one launch of the
+// forward's increment kernel) give segment g of a head the sum of segments
+// 0 .. g-1 as its carry-in; each CTA then walks its segment's chunks.
+//
+// The kernel is synchronous: 256 threads (8 warps, two per TMEM lane
+// quarter; "half" h = warp / 4 splits each phase's columns), thread 0 issues
+// a round of MMAs and commits them to one barrier that every thread waits
+// on. The state, the feature order and its doubled off-diagonal rows are
+// the forward's (psd_tc_common.cuh).
+//
+// Tensor memory (512 columns, fp32):
+//   [  0, 320)  S, five 128-feature tiles of 64 columns (tile 4: 16 rows used)
+//   [320, 352)  Z (lanes 0..31)
+//   [352, 384)  U = Q Z_c, then the dq accumulator
+//   [384, 512)  work: A | D' (64 keys each), or two 64-feature X blocks, or
+//               M (bf16) in the A columns
+#include "common.cuh"
+#include "launch.h"
+#include "profile.h"
+#include "tc_common.cuh"
+#include "tma_host.h"
+#include "psd_tc_common.cuh"
+
+namespace kata {
+namespace {
+
+using namespace tc;
+using namespace psd;
+
+constexpr int kBThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColZ = 320, kColDq = 352, kColA = 384, kColB = 448;
+
+// Shared memory (byte offsets from a 1024-aligned base).
+struct DqSmem {
+  static constexpr int Q = 0;                      // [128][32] bf16, 64-byte swizzle
+  static constexpr int K = 8192;                   // [128][32] bf16, 64-byte swizzle
+  static constexpr int V = 16384;                  // [128][64] bf16, 128-byte swizzle
+  static constexpr int dO = 32768;                 // [128][64] bf16, 128-byte swizzle
+  static constexpr int Snap = 49152;               // S_c bf16 [528][64], 128-byte rows
+  static constexpr int ZSnap = Snap + kD * 128;    // Z_c bf16 [32][32], 64-byte rows
+  static constexpr int Key = ZSnap + 2048;         // two key-feature tiles of 32 KB
+  static constexpr int Xch = Key + 2 * 32768;      // [128][36] fp32: half 1's partial sums
+  static constexpr int Ubuf = Xch + 128 * 36 * 4;  // [128][32] fp32: u = Z_c q
+  static constexpr int InvD = Ubuf + 128 * 32 * 4; // [128] fp32: 1 / d_t
+  static constexpr int Cc = InvD + 512;            // [128] fp32: c_t
+  static constexpr int Bars = Cc + 512;
+  static constexpr int Bytes = Bars + 64 + 1024;   // barriers + alignment slack
+  static_assert(Snap % 1024 == 0 && ZSnap % 1024 == 0 && Key % 1024 == 0, "swizzle atoms");
+  static_assert(Bytes <= 232448, "shared memory budget");
+};
+enum { kBarLoadQ = 0, kBarLoadKV, kBarMma, kNumBars };
+
+// One thread's q (or k) row as 32 fp32 values from a 64-byte-swizzled tile.
+__device__ __forceinline__ void row_f32(const uint8_t *tile, int row, float (&x)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4 *>(tile + sw64(row, c));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&w[j]);
+      x[8 * c + 2 * j] = __low2float(b);
+      x[8 * c + 2 * j + 1] = __high2float(b);
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void rot(float (&R)[32]) {
+  float t[32];
+#pragma unroll
+  for (int l = 0; l < 32; ++l) t[l] = R[(l + N) & 31];
+#pragma unroll
+  for (int l = 0; l < 32; ++l) R[l] = t[l];
+}
+
+// Contraction of one offset d of the feature order (features (l, (l+d) mod 32)
+// for l < nl) with its X values: x[l] = X_(d,l) (the state's doubled rows make
+// X_f = m_f (S dout)_f). qR = q rotated by d, g2R accumulates the Jacobian's
+// second term in the same rotated frame; both are rotated by one afterwards.
+template <int NL>
+__device__ __forceinline__ void contract_offset(const uint32_t *x, const float (&q)[32],
+                                                float (&qR)[32], float (&h)[32], float (&g2R)[32],
+                                                float &dn) {
+#pragma unroll
+  for (int l = 0; l < NL; ++l) {
+    const float xv = __uint_as_float(x[l]);
+    dn = fmaf(q[l] * qR[l], xv, dn);
+    h[l] = fmaf(qR[l], xv, h[l]);
+    g2R[l] = fmaf(q[l], xv, g2R[l]);
+  }
+  rot<1>(qR);
+  rot<1>(g2R);
+}
+
+__global__ void __launch_bounds__(kBThreads, 1)
+bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                 const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                 const float *__restrict__ aggS, __nv_bfloat16 *__restrict__ dq,
+                 float *__restrict__ den_out, float *__restrict__ c_out,
+                 unsigned *__restrict__ status, int T, int G, int seg_len) {
+  using L = DqSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::Bars);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::Bars + 8 * kNumBars);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::Bars + 8 * kNumBars + 4);
+  float *xch = reinterpret_cast<float *>(smem + L::Xch);
+  float *ubuf = reinterpret_cast<float *>(smem + L::Ubuf);
+  float *invd_s = reinterpret_cast<float *>(smem + L::InvD);
+  float *c_s = reinterpret_cast<float *>(smem + L::Cc);
+  uint8_t *snap = smem + L::Snap;
+  uint8_t *zsnap = smem + L::ZSnap;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int r = quarter * 32 + lane;                  // TMEM lane: token / feature row
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  const int g = blockIdx.x % G, bh = blockIdx.x / G;
+  const int t0 = g * seg_len, t1 = min(T, t0 + seg_len);
+  const int nchunks = (t1 - t0 + kC - 1) / kC;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kBarLoadQ], 1);
+    mbar_init(&bars[kBarLoadKV], 1);
+    mbar_init(&bars[kBarMma], 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  auto load_q = [&](int i) {        // Q and dout of chunk i
+    mbar_arrive_expect_tx(&bars[kBarLoadQ], 8192 + 16384);
+    tma_load_3d(smem + L::Q, &tmq, &bars[kBarLoadQ], 0, t0 + i * kC, bh);
+    tma_load_3d(smem + L::dO, &tmo, &bars[kBarLoadQ], 0, t0 + i * kC, bh);
+  };
+  auto load_kv = [&](int i) {       // K and V of chunk i
+    mbar_arrive_expect_tx(&bars[kBarLoadKV], 8192 + 16384);
+    tma_load_3d(smem + L::K, &tmk, &bars[kBarLoadKV], 0, t0 + i * kC, bh);
+    tma_load_3d(smem + L::V, &tmv, &bars[kBarLoadKV], 0, t0 + i * kC, bh);
+  };
+  if (threadIdx.x == 0 && nchunks > 0) {
+    tma_prefetch_desc(&tmq);
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+    tma_prefetch_desc(&tmo);
+    load_q(0);
+    load_kv(0);
+  }
+
+  // One synchronous round: every thread's operand writes (shared memory,
+  // tensor memory) and tensor-memory reads are complete, thread 0 issues the
+  // MMAs and commits them, every thread waits. The result is uniform over
+  // the CTA, so a timeout ends every thread's loop at the same point.
+  uint32_t mph = 0;
+  auto round = [&](auto issue) -> bool {
+    tmem_wait_ld();
+    tmem_wait_st();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue();
+      mma_commit(&bars[kBarMma]);
+    }
+    const bool ok = mbar_wait(&bars[kBarMma], mph, abort_flag);
+    mph ^= 1;
+    tc_fence_after();
+    return __syncthreads_and(ok);
+  };
+  auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+    return __syncthreads_and(mbar_wait(bar, parity, abort_flag));
+  };
+
+  // Descriptors (start-address field advanced by bytes / 16 for sub-tiles).
+  auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+  const uint64_t d_q = smem_desc(smem_u32(smem + L::Q), 16, 512, kSw64);          // K-major
+  const uint64_t d_k = smem_desc(smem_u32(smem + L::K), 16, 512, kSw64);          // K-major
+  const uint64_t d_k_mn = smem_desc(smem_u32(smem + L::K), 8192, 512, kSw64);     // MN-major
+  const uint64_t d_v = smem_desc(smem_u32(smem + L::V), 16, 1024, kSw128);        // K-major
+  const uint64_t d_v_mn = smem_desc(smem_u32(smem + L::V), 16384, 1024, kSw128);  // MN-major
+  const uint64_t d_o = smem_desc(smem_u32(smem + L::dO), 16, 1024, kSw128);       // K-major
+  const uint64_t d_snap = smem_desc(smem_u32(snap), 16, 1024, kSw128);            // K-major
+  const uint64_t d_z = smem_desc(smem_u32(zsnap), 16, 512, kSw64);
+  const uint64_t d_key = smem_desc(smem_u32(smem + L::Key), 16384, 1024, kSw128); // MN-major
+  constexpr uint32_t id_n64 = idesc_bf16(128, 64, false, false);
+  constexpr uint32_t id_n32 = idesc_bf16(128, 32, false, false);
+  constexpr uint32_t id_n16 = idesc_bf16(128, 16, false, false);
+  constexpr uint32_t id_mk = idesc_bf16(128, 32, false, true);      // M (TMEM) x K_b (MN-major)
+  constexpr uint32_t id_up = idesc_bf16(128, 64, true, true);
+  constexpr uint32_t id_z = idesc_bf16(128, 32, true, true);
+
+  // A = Q K_b^T and D' = dout V_b^T for keys 64 b .. 64 b + 63
+  auto issue_intra = [&](int b) {
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk)
+      mma_ss(tbase + kColA, adv(d_q, 32 * kk), adv(d_k, 4096 * b + 32 * kk), id_n64, kk);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_v, 8192 * b + 32 * kk), id_n64, kk);
+  };
+
+  // ---- carry-in: S, Z = the increments of segments 0 .. g-1 ----
+  {
+    const float *seg0 = aggS + (size_t)bh * G * kAggFloats;
+    // half 0: tiles 0, 1 and 4; half 1: tiles 2, 3 and Z
+    for (int m = half ? 2 : 0; m < (half ? 4 : 2) + (half ? 0 : 1); ++m) {
+      const int mt = (!half && m == 2) ? 4 : m;
+      const int f = 128 * mt + r;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float acc[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+        if (f < kD) {
+          for (int gp = 0; gp < g; ++gp) {
+            const float4 *src =
+                reinterpret_cast<const float4 *>(seg0 + (size_t)gp * kAggFloats + f * kDV + 16 * q4);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const float4 x = src[c4];
+              acc[4 * c4 + 0] += x.x;
+              acc[4 * c4 + 1] += x.y;
+              acc[4 * c4 + 2] += x.z;
+              acc[4 * c4 + 3] += x.w;
+            }
+          }
+        }
+        uint32_t bits[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) bits[c] = __float_as_uint(acc[c]);
+        tmem_st16(tbase + lane_off + kColS + 64 * mt + 16 * q4, bits);
+        if (f < kD) {
+          *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4)) = pack8(bits);
+          *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4 + 1)) = pack8(bits + 8);
+        }
+      }
+    }
+    if (half) {
+      float acc[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+      if (r < kDK) {
+        for (int gp = 0; gp < g; ++gp) {
+          const float4 *src =
+              reinterpret_cast<const float4 *>(seg0 + (size_t)gp * kAggFloats + kD * kDV + r * kDK);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 x = src[c4];
+            acc[4 * c4 + 0] += x.x;
+            acc[4 * c4 + 1] += x.y;
+            acc[4 * c4 + 2] += x.z;
+            acc[4 * c4 + 3] += x.w;
+          }
+        }
+      }
+      uint32_t bits[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) bits[c] = __float_as_uint(acc[c]);
+      tmem_st32(tbase + lane_off + kColZ, bits);
+      if (quarter == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(zsnap + sw64(r, c)) = pack8(bits + 8 * c);
+      }
+    }
+  }
+
+  bool ok = true;
+  for (int i = 0; ok && i < nchunks; ++i) {
+    const int c0 = t0 + i * kC;
+    const bool valid = c0 + r < T;
+    if (!(ok = wait_all(&bars[kBarLoadQ], i & 1) && wait_all(&bars[kBarLoadKV], i & 1))) break;
+    float q[32];
+    row_f32(smem + L::Q, r, q);
+
+    // ---- intra-chunk row sums: l = sum_s w_ts, dn = sum_s w_ts (dout_t . v_s) ----
+    float l_part = 0.f, dn_part = 0.f, den_inter = 0.f;
+    for (int b = 0; ok && b < 2; ++b) {
+      ok = round([&] {
+        if (b == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_ss(tbase + kColDq, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_n32, kk);
+        }
+        issue_intra(b);
+      });
+      if (!ok) break;
+      uint32_t a[32], dp[32];
+      tmem_ld32(tbase + lane_off + kColA + 32 * half, a);
+      tmem_ld32(tbase + lane_off + kColB + 32 * half, dp);
+      tmem_wait_ld();
+      const int s0 = 64 * b + 32 * half;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float av = __uint_as_float(a[j]);
+        const float w = s0 + j <= r ? av * av : 0.f;
+        l_part += w;
+        dn_part = fmaf(w, __uint_as_float(dp[j]), dn_part);
+      }
+      if (b == 0 && half == 0) {
+        // u = Z_c q: the carried denominator q^T Z_c q, and 2 c_t u for dq
+        uint32_t u[32];
+        tmem_ld32(tbase + lane_off + kColDq, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) den_inter = fmaf(q[j], __uint_as_float(u[j]), den_inter);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4 *>(ubuf + r * 32 + j) =
+              make_float4(__uint_as_float(u[j]), __uint_as_float(u[j + 1]),
+                          __uint_as_float(u[j + 2]), __uint_as_float(u[j + 3]));
+      }
+    }
+    if (!ok) break;
+
+    // ---- carried part: X = dout S_c^T, 64 features a round and half ----
+    // half 0 takes features 0 .. 255 (offsets d = 0 .. 7), half 1 features
+    // 256 .. 527 (d = 8 .. 15 and the 16 pairs (l, l + 16)).
+    float h[32], g2R[32], qR[32];
+#pragma unroll
+    for (int l = 0; l < 32; ++l) {
+      h[l] = 0.f;
+      g2R[l] = 0.f;
+      qR[l] = q[l];
+    }
+    if (half) rot<8>(qR);
+    float dn_car = 0.f;
+    for (int j = 0; ok && j < 5; ++j) {
+      ok = round([&] {
+        if (j < 4) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tbase + kColA, adv(d_o, 32 * kk), adv(d_snap, 64 * j * 128 + 32 * kk), id_n64, kk);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_snap, (256 + 64 * j) * 128 + 32 * kk),
+                   id_n64, kk);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
+        }
+      });
+      if (!ok) break;
+      if (j < 4) {
+        uint32_t x[32];
+        tmem_ld32(tbase + lane_off + kColA + 64 * half, x);
+        tmem_wait_ld();
+        contract_offset<32>(x, q, qR, h, g2R, dn_car);
+        tmem_ld32(tbase + lane_off + kColA + 64 * half + 32, x);
+        tmem_wait_ld();
+        contract_offset<32>(x, q, qR, h, g2R, dn_car);
+      } else if (half) {
+        uint32_t x[16];
+        tmem_ld16(tbase + lane_off + kColB, x);
+        tmem_wait_ld();
+        contract_offset<16>(x, q, qR, h, g2R, dn_car);
+      }
+    }
+    if (!ok) break;
+    // back to the unrotated frame: half 0 ended at offset 8, half 1 at 17
+    if (half) {
+      rot<15>(g2R);
+    } else {
+      rot<24>(g2R);
+    }
+#pragma unroll
+    for (int l = 0; l < 32; ++l) h[l] += g2R[l];
+
+    // ---- combine the halves: d_t, c_t, the carried dq ----
+    if (half) {
+      float *row = xch + r * 36;
+      row[32] = l_part;
+      row[33] = dn_part + dn_car;
+#pragma unroll
+      for (int l = 0; l < 32; l += 4)
+        *reinterpret_cast<float4 *>(row + l) = make_float4(h[l], h[l + 1], h[l + 2], h[l + 3]);
+    }
+    __syncthreads();
+    float dqc[32];
+    if (!half) {
+      const float *row = xch + r * 36;
+      const float l_all = l_part + row[32];
+      const float dn_all = dn_part + dn_car + row[33];
+      const float d = l_all + den_inter;
+      if (valid && !(d > 0.f)) flag_status(status, kStatusNonPositiveNormaliser);
+      const float inv = valid ? 1.f / d : 0.f;
+      const float ct = valid ? -dn_all * inv * inv : 0.f;
+      invd_s[r] = inv;
+      c_s[r] = ct;
+      if (valid) {
+        den_out[(size_t)bh * T + c0 + r] = d;
+        c_out[(size_t)bh * T + c0 + r] = ct;
+      }
+      const float *u = ubuf + r * 32;
+#pragma unroll
+      for (int l = 0; l < 32; ++l) dqc[l] = inv * (h[l] + row[l]) + 2.f * ct * u[l];
+    }
+    __syncthreads();
+
+    // ---- intra-chunk dq: M = 2 A (D' / d_t + c_t) masked, dq += M K_b ----
+    const float inv_r = invd_s[r], c_r = c_s[r];
+    for (int b = 0; ok && b < 2; ++b) {
+      ok = round([&] { issue_intra(b); });
+      if (!ok) break;
+      if (b == 1 && threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);   // Q, dout read
+      uint32_t a[32], dp[32], m[16];
+      tmem_ld32(tbase + lane_off + kColA + 32 * half, a);
+      tmem_ld32(tbase + lane_off + kColB + 32 * half, dp);
+      tmem_wait_ld();
+      const int s0 = 64 * b + 32 * half;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float a0 = __uint_as_float(a[2 * j]), a1 = __uint_as_float(a[2 * j + 1]);
+        const float e0 = fmaf(__uint_as_float(dp[2 * j]), inv_r, c_r);
+        const float e1 = fmaf(__uint_as_float(dp[2 * j + 1]), inv_r, c_r);
+        const float m0 = s0 + 2 * j <= r ? 2.f * a0 * e0 : 0.f;
+        const float m1 = s0 + 2 * j + 1 <= r ? 2.f * a1 * e1 : 0.f;
+        m[j] = pack_bf16x2(m0, m1);
+      }
+      __syncthreads();          // every thread has read A and D' before M overwrites A
+      tmem_st16(tbase + lane_off + kColA + 16 * half, m);
+      ok = round([&] {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tbase + kColDq, tbase + kColA + 8 * kk, adv(d_k_mn, 4096 * b + 1024 * kk), id_mk,
+                 (b > 0 || kk > 0) ? 1u : 0u);
+      });
+    }
+    if (!ok) break;
+    if (!half) {
+      uint32_t acc[32];
+      tmem_ld32(tbase + lane_off + kColDq, acc);
+      tmem_wait_ld();
+      if (valid) {
+        uint4 *dst = reinterpret_cast<uint4 *>(dq + ((size_t)bh * T + c0 + r) * kDK);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            w[j] = pack_bf16x2(__uint_as_float(acc[8 * c + 2 * j]) + dqc[8 * c + 2 * j],
+                               __uint_as_float(acc[8 * c + 2 * j + 1]) + dqc[8 * c + 2 * j + 1]);
+          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    if (i == nchunks - 1) break;            // the state after the segment is not needed
+
+    // ---- update: S += phi(K)^T V, Z += K^T K; three rounds of two key tiles ----
+    {
+      uint32_t XK[16], P[32], R2[32];
+      load_pairs(smem + L::K, r, XK, P);
+#pragma unroll
+      for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[l], 0x40004000u);   // x 2.0
+      // tiles: round 0 (0, 2), round 1 (1, 3), round 2 (4, -)
+      if (half) rotate_left(R2, 8);
+      for (int u = 0; ok && u < 3; ++u) {
+        const int m = half ? (u < 2 ? 2 + u : -1) : (u < 2 ? u : 4);
+        if (m >= 0)
+          write_tile(smem + L::Key + 32768 * half, r, m == kTiles - 1,
+                     m == 0 ? 0x3f003f00u : 0x3f803f80u, P, R2);
+        if (!half && u == 1) {
+          rotate_left(R2, 12);
+        } else {
+          rotate_left(R2, 4);
+        }
+        ok = round([&] {
+          const int ma = u < 2 ? u : 4, mb = 2 + u;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tbase + kColS + 64 * ma, adv(d_key, 2048 * kk), adv(d_v_mn, 2048 * kk), id_up, 1);
+          if (u < 2) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + kColS + 64 * mb, adv(d_key, 32768 + 2048 * kk), adv(d_v_mn, 2048 * kk),
+                     id_up, 1);
+          }
+          if (u == 0) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + kColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1);
+          }
+        });
+      }
+      if (!ok) break;
+      if (threadIdx.x == 0) load_kv(i + 1);           // K, V of this chunk no longer read
+    }
+    // ---- snapshot S_c+1 (half 0: tiles 0, 1, 4; half 1: tiles 2, 3) and Z_c+1 ----
+    for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
+      const int mt = (!half && m == 2) ? 4 : m;
+      if (mt == 4 && quarter != 0) continue;        // tile 4: rows 512..527 (lanes 0..15)
+      const int f = 128 * mt + r;
+      uint32_t a[32], b2[32];
+      tmem_ld32(tbase + lane_off + kColS + 64 * mt, a);
+      tmem_ld32(tbase + lane_off + kColS + 64 * mt + 32, b2);
+      tmem_wait_ld();
+      if (f < kD) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          *reinterpret_cast<uint4 *>(snap + sw128(f, q4)) = pack8(a + 8 * q4);
+          *reinterpret_cast<uint4 *>(snap + sw128(f, 4 + q4)) = pack8(b2 + 8 * q4);
+        }
+      }
+    }
+    if (half && quarter == 0) {
+      uint32_t zr[32];
+      tmem_ld32(tbase + lane_off + kColZ, zr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(zsnap + sw64(r, c)) = pack8(zr + 8 * c);
+    }
+  }
+  if (*abort_flag && threadIdx.x == 0) flag_status(status, kStatusDeviceTimeout);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t tc_bwd_dq(const BackwardLaunch &a, float *aggS, int G, int seg_len) {
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tma_3d_bf16(&tq, a.q, kDK, a.T, a.BH, kC) ||
+      !make_tma_3d_bf16(&tk, a.k, kDK, a.T, a.BH, kC) ||
+      !make_tma_3d_bf16(&tv, a.v, kDV, a.T, a.BH, kC) ||
+      !make_tma_3d_bf16(&to, a.dout, kDV, a.T, a.BH, kC))
+    return cudaErrorInvalidValue;
+  cudaError_t e = psd_tc_increments(a.k, a.v, aggS, a.status, a.BH, a.T, G - 1, G, seg_len, a.stream);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           DqSmem::Bytes);
+  if (e != cudaSuccess) return e;
+  ProfileScope prof("tc_bwd_dq", a.stream);
+  bwd_dq_tc_kernel<<<(unsigned)(a.BH * G), kBThreads, DqSmem::Bytes, a.stream>>>(
+      tq, tk, tv, to, aggS, static_cast<__nv_bfloat16 *>(a.dq), a.den, a.c, a.status, a.T, G,
+      seg_len);
+  return cudaGetLastError();
+}
+
+}  // namespace kata

@@ -789,6 +789,33 @@ void tc_chunked_layout(long long BH, int T, int sms, bool sequential, int *G, in
   *P = 1;
 }
 
+namespace {
+// Launches the increment kernel over segments 0 .. G_inc - 1 (grid of BH x
+// G_inc CTAs; agg strided by G_total increments per head).
+cudaError_t launch_increments(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                              const CUtensorMap &to, float *agg, unsigned *status, long long BH,
+                              int T, int G_inc, int G_total, int seg_len, cudaStream_t stream) {
+  auto kagg = chunked_tc_kernel<true>;
+  cudaError_t e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Layout<true>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  ProfileScope prof("tc_segment_increment", stream);
+  kagg<<<(unsigned)(BH * G_inc), kThreads, Layout<true>::kSmemBytes, stream>>>(
+      tq, tk, tv, to, agg, nullptr, nullptr, nullptr, nullptr, status, T, G_inc, G_total, seg_len);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t psd_tc_increments(const void *k, const void *v, float *agg, unsigned *status,
+                              long long BH, int T, int G_inc, int G_total, int seg_len,
+                              cudaStream_t stream) {
+  if (G_inc <= 0) return cudaSuccess;
+  CUtensorMap tk, tv;
+  if (!make_tma_3d_bf16(&tk, k, kDK, T, BH, kC) || !make_tma_3d_bf16(&tv, v, kDV, T, BH, kC))
+    return cudaErrorInvalidValue;
+  return launch_increments(tk, tk, tv, tv, agg, status, BH, T, G_inc, G_total, seg_len, stream);
+}
+
 cudaError_t tc_chunked(const ChunkedLaunch &a) {
   int G, seg_len, P;
   tc_chunked_layout(a.BH, a.T, a.sms, a.sequential, &G, &seg_len, &P);
@@ -803,18 +830,10 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
   cudaError_t e;
   // increments of segments 0 .. G-2 (all G for the state-only call)
   const int G_inc = a.state_only ? G : G - 1;
-  if (G_inc > 0) {
-    auto kagg = chunked_tc_kernel<true>;
-    e = cudaFuncSetAttribute(kagg, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Layout<true>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    ProfileScope prof("tc_segment_increment", a.stream);
-    kagg<<<(unsigned)(a.BH * G_inc), kThreads, Layout<true>::kSmemBytes, a.stream>>>(
-        tq, tk, tv, to, a.agg, nullptr, nullptr, nullptr, nullptr, a.status, a.T, G_inc, G,
-        seg_len);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  if (G_inc > 0 &&
+      (e = launch_increments(tq, tk, tv, to, a.agg, a.status, a.BH, a.T, G_inc, G, seg_len,
+                             a.stream)) != cudaSuccess)
+    return e;
   if (a.state_only)
     return state_reduce(kAggPsdTc, a.agg, a.BH, G, kD, kDK, kDV, a.S_out, a.z_out, 0.f, a.stream);
   auto kpass = chunked_tc_kernel<false>;

@@ -95,9 +95,28 @@ struct BwdLayout {
   size_t total() const { return kHeaderBytes + 2 * agg_bytes + 2 * den_bytes; }
 };
 
-BwdLayout bwd_layout(long long BH, int T, int D, int d_v, const Split &sp) {
-  return {align_up((size_t)BH * (size_t)sp.G * (size_t)D * (size_t)(d_v + 1) * sizeof(float), kAlign),
-          align_up((size_t)BH * (size_t)T * sizeof(float), kAlign)};
+// The tensor-core dq pass (bf16 PSD, d_k = 32, d_v = 64) keeps its prefix
+// increments in the forward's tensor-core layout and split; each increment
+// region is sized for the larger of the two layouts.
+bool bwd_tc_shape(int d_k, int d_v, int C, kata_dtype_t dtype, kata_feature_t feature) {
+  return dtype == KATA_DTYPE_BF16 && feature == KATA_FEATURE_PSD && d_k == 32 && d_v == 64 &&
+         (C == 64 || C == 128);
+}
+
+void bwd_tc_split(long long BH, int T, int sms, int *G, int *seg_len) {
+  int P;
+  tc_chunked_layout(BH, T, sms, false, G, seg_len, &P);
+}
+
+BwdLayout bwd_layout(long long BH, int T, int D, int d_v, const Split &sp, bool tc, int sms) {
+  size_t agg = (size_t)BH * (size_t)sp.G * (size_t)D * (size_t)(d_v + 1) * sizeof(float);
+  if (tc) {
+    int G, seg_len;
+    bwd_tc_split(BH, T, sms, &G, &seg_len);
+    const size_t tc_agg = (size_t)BH * (size_t)G * tc_chunked_agg_floats() * sizeof(float);
+    agg = agg > tc_agg ? agg : tc_agg;
+  }
+  return {align_up(agg, kAlign), align_up((size_t)BH * (size_t)T * sizeof(float), kAlign)};
 }
 
 // Calls F::template run<DK, DV, FEAT>() for the runtime (d_k, d_v, feature).
@@ -178,9 +197,19 @@ struct BackwardRun {
   static constexpr bool kBaseFeaturesOnly = true;     // the gradient covers PSD and first-order
   kata_dtype_t dtype;
   BackwardLaunch a;
+  bool tc;                 // bf16 PSD d_k = 32, d_v = 64: the tensor-core dq pass
+  int tc_G, tc_seg_len;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
-    const cudaError_t e = dtype == KATA_DTYPE_F32 ? simt_backward<DK, DV, FEAT, float>(a)
-                                                  : simt_backward<DK, DV, FEAT, __nv_bfloat16>(a);
+    cudaError_t e;
+    if constexpr (DK == 32 && DV == 64 && FEAT == kPSD) {
+      if (tc) {
+        e = tc_bwd_dq(a, a.aggS, tc_G, tc_seg_len);
+        if (e == cudaSuccess) e = simt_backward_dkdv<DK, DV, FEAT, __nv_bfloat16>(a);
+        return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+      }
+    }
+    e = dtype == KATA_DTYPE_F32 ? simt_backward<DK, DV, FEAT, float>(a)
+                                : simt_backward<DK, DV, FEAT, __nv_bfloat16>(a);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
   }
 };
@@ -396,7 +425,9 @@ size_t kata_bwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, i
   if (sms <= 0) return 0;
   const long long BH = (long long)B * H;
   const Split sp = segment_split(BH, T, C, sms, false);
-  return bwd_layout(BH, T, (int)kata_state_dim(d_k, feature), d_v, sp).total();
+  return bwd_layout(BH, T, (int)kata_state_dim(d_k, feature), d_v, sp,
+                    bwd_tc_shape(d_k, d_v, C, dtype, feature), sms)
+      .total();
 }
 
 kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
@@ -414,20 +445,29 @@ kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
   if (sms <= 0) return KATA_ERR_CUDA;
   const long long BH = (long long)B * H;
   const Split sp = segment_split(BH, T, C, sms, false);
-  const BwdLayout lay = bwd_layout(BH, T, (int)kata_state_dim(d_k, feature), d_v, sp);
+  const bool tc_shape = bwd_tc_shape(d_k, d_v, C, dtype, feature);
+  const BwdLayout lay = bwd_layout(BH, T, (int)kata_state_dim(d_k, feature), d_v, sp, tc_shape, sms);
   if (workspace_bytes < lay.total()) return KATA_ERR_WORKSPACE;
   unsigned char *ws = static_cast<unsigned char *>(workspace);
   if (cudaMemsetAsync(ws, 0, sizeof(unsigned), stream) != cudaSuccess) return KATA_ERR_CUDA;
   if (BH == 0 || T == 0) return KATA_OK;
   if (!q || !k || !v || !dout || !dq || !dk || !dv) return KATA_ERR_INVALID_ARGUMENT;
   if (BH * (long long)sp.G > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
-  BackwardRun run{dtype, BackwardLaunch{q, k, v, dout, dq, dk, dv, BH, T,
-                                        reinterpret_cast<unsigned *>(ws),
-                                        reinterpret_cast<float *>(ws + lay.aggS()),
-                                        reinterpret_cast<float *>(ws + lay.aggR()),
-                                        reinterpret_cast<float *>(ws + lay.den()),
-                                        reinterpret_cast<float *>(ws + lay.c()), sp.G, sp.seg_len,
-                                        stream}};
+  // the tensor-core pass reads its operands by TMA and writes dq rows as
+  // 16-byte vectors: 16-byte aligned pointers
+  bool tc = tc_shape;
+  for (const void *p : {q, k, v, dout, (const void *)dq})
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0) tc = false;
+  int tc_G = 1, tc_seg_len = T;
+  if (tc) bwd_tc_split(BH, T, sms, &tc_G, &tc_seg_len);
+  BackwardRun run{dtype,
+                  BackwardLaunch{q, k, v, dout, dq, dk, dv, BH, T,
+                                 reinterpret_cast<unsigned *>(ws),
+                                 reinterpret_cast<float *>(ws + lay.aggS()),
+                                 reinterpret_cast<float *>(ws + lay.aggR()),
+                                 reinterpret_cast<float *>(ws + lay.den()),
+                                 reinterpret_cast<float *>(ws + lay.c()), sp.G, sp.seg_len, stream},
+                  tc, tc_G, tc_seg_len};
   return dispatch_shape(d_k, d_v, feature, run);
 }
 

@@ -106,6 +106,17 @@ cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature
 bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t tc_chunked(const ChunkedLaunch &a);
 size_t tc_chunked_agg_floats();   // floats of one segment increment
+// Tensor-core gradient with respect to q of the PSD chunked forward (bf16,
+// d_k = 32, d_v = 64): the forward's increments of segments 0 .. G-2 into
+// aggS (PSD tensor-core layout, G per head), then dq and, per token, d_t and
+// c_t (a.den, a.c) for the suffix pass; G segments of seg_len tokens.
+cudaError_t tc_bwd_dq(const BackwardLaunch &a, float *aggS, int G, int seg_len);
+// Segment increments of the PSD tensor-core layout (d_k = 32, d_v = 64 bf16):
+// segments 0 .. G_inc - 1 of G_total (seg_len tokens each, whole 128-token
+// chunks) into agg[bh][g], G_total increments per head.
+cudaError_t psd_tc_increments(const void *k, const void *v, float *agg, unsigned *status,
+                              long long BH, int T, int G_inc, int G_total, int seg_len,
+                              cudaStream_t stream);
 // The PSD tensor-core forward's split: G segments of seg_len tokens per head,
 // each segment's increment computed as P pieces (G * P increments per head in
 // the workspace).
@@ -122,5 +133,7 @@ template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_chunked(const
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_quadratic(const QuadraticLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_decode(const DecodeLaunch &a);
 template <int DK, int DV, int FEAT, typename Tin> cudaError_t simt_backward(const BackwardLaunch &a);
+template <int DK, int DV, int FEAT, typename Tin>
+cudaError_t simt_backward_dkdv(const BackwardLaunch &a);
 
 }  // namespace kata

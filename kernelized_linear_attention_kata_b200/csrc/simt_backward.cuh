@@ -600,6 +600,36 @@ bwd_dkdv_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
   }
 }
 
+// The suffix half of the backward (launches 3 and 4): the suffix-state
+// increments and the dk, dv walk, from the d_t and c_t of the dq pass.
+template <int DK, int DV, int FEAT, typename Tin>
+cudaError_t simt_backward_dkdv(const BackwardLaunch &a) {
+  constexpr int D = state_dim(DK, FEAT);
+  const Tin *q = static_cast<const Tin *>(a.q);
+  const Tin *k = static_cast<const Tin *>(a.k);
+  const Tin *v = static_cast<const Tin *>(a.v);
+  const Tin *dy = static_cast<const Tin *>(a.dout);
+  const int inc_threads = (D + 31) / 32 * 32;
+  constexpr size_t smem = BwdSmem<DK, DV, FEAT>::bytes;
+  cudaError_t e;
+  if (a.G > 1) {
+    ProfileScope prof("simt_bwd_suffix_increment", a.stream);
+    bwd_increment_kernel<DK, DV, FEAT, Tin>
+        <<<(unsigned)(a.BH * (a.G - 1)), inc_threads, 0, a.stream>>>(q, dy, a.den, a.c, a.aggR, a.T,
+                                                                      a.G, a.seg_len);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  auto kern = bwd_dkdv_kernel<DK, DV, FEAT, Tin>;
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+      cudaSuccess)
+    return e;
+  ProfileScope prof("simt_bwd_dkdv", a.stream);
+  kern<<<(unsigned)(a.BH * a.G), kBwdThreads, smem, a.stream>>>(
+      q, k, v, dy, static_cast<Tin *>(a.dk), static_cast<Tin *>(a.dv), a.aggR, a.den, a.c, a.T, a.G,
+      a.seg_len);
+  return cudaGetLastError();
+}
+
 template <int DK, int DV, int FEAT, typename Tin>
 cudaError_t simt_backward(const BackwardLaunch &a) {
   constexpr int D = state_dim(DK, FEAT);
@@ -627,25 +657,11 @@ cudaError_t simt_backward(const BackwardLaunch &a) {
         q, k, v, dy, static_cast<Tin *>(a.dq), a.aggS, a.den, a.c, a.status, a.T, a.G, a.seg_len);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if (a.G > 1) {
-    ProfileScope prof("simt_bwd_suffix_increment", a.stream);
-    bwd_increment_kernel<DK, DV, FEAT, Tin>
-        <<<(unsigned)(a.BH * (a.G - 1)), inc_threads, 0, a.stream>>>(q, dy, a.den, a.c, a.aggR, a.T,
-                                                                      a.G, a.seg_len);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  auto kern = bwd_dkdv_kernel<DK, DV, FEAT, Tin>;
-  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-      cudaSuccess)
-    return e;
-  ProfileScope prof("simt_bwd_dkdv", a.stream);
-  kern<<<(unsigned)(a.BH * a.G), kBwdThreads, smem, a.stream>>>(
-      q, k, v, dy, static_cast<Tin *>(a.dk), static_cast<Tin *>(a.dv), a.aggR, a.den, a.c, a.T, a.G,
-      a.seg_len);
-  return cudaGetLastError();
+  return simt_backward_dkdv<DK, DV, FEAT, Tin>(a);
 }
 
-#define KATA_INSTANTIATE_BACKWARD(DK, DV, FEAT, TIN) \
-  template cudaError_t simt_backward<DK, DV, FEAT, TIN>(const BackwardLaunch &);
+#define KATA_INSTANTIATE_BACKWARD(DK, DV, FEAT, TIN)                              \
+  template cudaError_t simt_backward<DK, DV, FEAT, TIN>(const BackwardLaunch &);    \
+  template cudaError_t simt_backward_dkdv<DK, DV, FEAT, TIN>(const BackwardLaunch &);
 
 }  // namespace kata
