@@ -555,6 +555,568 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
   if (warp == 0) tmem_dealloc(tbase, kTmemCols);
 }
 
+// ---------------------------------------------------------------------------
+// The suffix pass: dk and dv, chunks in reverse order.
+//
+// With the suffix state R = sum_(t in later chunks) phi_q(q_t) g_t^T and
+// Rq = sum c_t q_t q_t^T (so that r . phi(k) = k^T Rq k):
+//   dv_s (carried) = R^T phi(k_s),
+//   dk_s (carried) = J(k_s)^T (R v_s) + 2 Rq k_s,
+//   dv_s (intra)   = sum_(t>=s) w_ts g_t,
+//   dk_s (intra)   = sum_(t>=s) e_ts 2 (q_t . k_s) q_t,
+// then R += phi_q(Q_c)^T G_c, Rq += Q_c^T diag(c) Q_c. R is held with the
+// off-diagonal rows doubled (R'_f = m_f R_f), as the forward holds S, so that
+// plain key products read it out.
+//
+// Tensor memory (512 columns, fp32):
+//   [  0, 320)  R', five 128-feature tiles
+//   [320, 352)  Rq (lanes 0..31)
+//   [352, 384)  U2 = K Rq, then the dk accumulator
+//   [384, 448)  the dv accumulator (first a 64-feature Y block of half 0)
+//   [448, 512)  work: a Y block of half 1; K Q^T | V dout^T (32 queries
+//               each); W~ | M (bf16)
+// The increment kernel (AGG) runs only the update over its segment and
+// writes the segment's (R', Rq) increment.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kColR = 0, kColRq = 320, kColDk = 352, kColDv = 384, kColW = 448;
+constexpr int kQSlotsPsd = 9;      // 64-feature slots of the readout (the last holds 16)
+
+struct DkvSmem {
+  static constexpr int Q = 0;
+  static constexpr int K = 8192;
+  static constexpr int V = 16384;
+  static constexpr int dO = 32768;
+  static constexpr int Snap = 49152;                 // R' bf16 [528][64]
+  static constexpr int RqSnap = Snap + kD * 128;     // Rq bf16 [32][32]
+  static constexpr int Slots = RqSnap + 2048;        // 2 x 16 KB key-product slots, or
+                                                     // 2 x 32 KB query-feature tiles
+  static constexpr int CQ = Slots + 2 * 32768;       // [128][32] bf16 c_t q_t, 64-byte swizzle
+  static constexpr int Xch = CQ + 8192;              // [128][36] fp32
+  static constexpr int Ubuf = Xch + 128 * 36 * 4;    // [128][32] fp32: Rq k
+  static constexpr int InvD = Ubuf + 128 * 32 * 4;
+  static constexpr int Cc = InvD + 512;
+  static constexpr int Bars = Cc + 512;
+  static constexpr int Bytes = Bars + 64 + 1024;
+  static_assert(Snap % 1024 == 0 && RqSnap % 1024 == 0 && Slots % 1024 == 0 && CQ % 1024 == 0,
+                "swizzle atoms");
+  // the Rq update's A operand (M = 128 over a 32-row tile) reads three more
+  // 8 KB atoms past CQ: they must lie inside the allocation
+  static_assert(CQ + 4 * 8192 <= Bars, "padded A rows of the Rq update");
+  static_assert(Bytes <= 232448, "shared memory budget");
+};
+
+template <bool AGG>
+__global__ void __launch_bounds__(kBThreads, 1)
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                   float *__restrict__ aggR, const float *__restrict__ den,
+                   const float *__restrict__ cvec, __nv_bfloat16 *__restrict__ dk,
+                   __nv_bfloat16 *__restrict__ dv, unsigned *__restrict__ status, int T, int G,
+                   int seg_len) {
+  using L = DkvSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::Bars);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::Bars + 8 * kNumBars);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::Bars + 8 * kNumBars + 4);
+  float *xch = reinterpret_cast<float *>(smem + L::Xch);
+  float *ubuf = reinterpret_cast<float *>(smem + L::Ubuf);
+  float *invd_s = reinterpret_cast<float *>(smem + L::InvD);
+  float *c_s = reinterpret_cast<float *>(smem + L::Cc);
+  uint8_t *snap = smem + L::Snap;
+  uint8_t *rqsnap = smem + L::RqSnap;
+  uint8_t *slots = smem + L::Slots;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int r = quarter * 32 + lane;
+  const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+  // the increment kernel covers segments 1 .. G-1 (the carry of the earlier ones)
+  const int G_grid = AGG ? G - 1 : G;
+  const int g = blockIdx.x % G_grid + (AGG ? 1 : 0), bh = blockIdx.x / G_grid;
+  const int t0 = g * seg_len, t1 = min(T, t0 + seg_len);
+  const int nchunks = (t1 - t0 + kC - 1) / kC;
+  // chunk order: the pass walks backwards, the increment kernel forwards
+  auto chunk_of = [&](int i) { return AGG ? i : nchunks - 1 - i; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kBarLoadQ], 1);
+    mbar_init(&bars[kBarLoadKV], 1);
+    mbar_init(&bars[kBarMma], 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  auto load_q = [&](int i) {        // Q and dout of the i-th chunk in walk order
+    const int row = t0 + chunk_of(i) * kC;
+    mbar_arrive_expect_tx(&bars[kBarLoadQ], 8192 + 16384);
+    tma_load_3d(smem + L::Q, &tmq, &bars[kBarLoadQ], 0, row, bh);
+    tma_load_3d(smem + L::dO, &tmo, &bars[kBarLoadQ], 0, row, bh);
+  };
+  auto load_kv = [&](int i) {
+    const int row = t0 + chunk_of(i) * kC;
+    mbar_arrive_expect_tx(&bars[kBarLoadKV], 8192 + 16384);
+    tma_load_3d(smem + L::K, &tmk, &bars[kBarLoadKV], 0, row, bh);
+    tma_load_3d(smem + L::V, &tmv, &bars[kBarLoadKV], 0, row, bh);
+  };
+  if (threadIdx.x == 0 && nchunks > 0) {
+    tma_prefetch_desc(&tmq);
+    tma_prefetch_desc(&tmo);
+    load_q(0);
+    if (!AGG) {
+      tma_prefetch_desc(&tmk);
+      tma_prefetch_desc(&tmv);
+      load_kv(0);
+    }
+  }
+
+  uint32_t mph = 0;
+  auto round = [&](auto issue) -> bool {
+    tmem_wait_ld();
+    tmem_wait_st();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue();
+      mma_commit(&bars[kBarMma]);
+    }
+    const bool ok = mbar_wait(&bars[kBarMma], mph, abort_flag);
+    mph ^= 1;
+    tc_fence_after();
+    return __syncthreads_and(ok);
+  };
+  auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
+    return __syncthreads_and(mbar_wait(bar, parity, abort_flag));
+  };
+
+  auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+  const uint64_t d_q = smem_desc(smem_u32(smem + L::Q), 16, 512, kSw64);          // K-major
+  const uint64_t d_q_mn = smem_desc(smem_u32(smem + L::Q), 8192, 512, kSw64);     // MN-major
+  const uint64_t d_k = smem_desc(smem_u32(smem + L::K), 16, 512, kSw64);          // K-major
+  const uint64_t d_v = smem_desc(smem_u32(smem + L::V), 16, 1024, kSw128);        // K-major
+  const uint64_t d_o = smem_desc(smem_u32(smem + L::dO), 16, 1024, kSw128);       // K-major
+  const uint64_t d_o_mn = smem_desc(smem_u32(smem + L::dO), 16384, 1024, kSw128); // MN-major
+  const uint64_t d_snap = smem_desc(smem_u32(snap), 16, 1024, kSw128);            // K-major
+  const uint64_t d_snap_mn = smem_desc(smem_u32(snap), 16384, 1024, kSw128);      // MN-major
+  const uint64_t d_rq = smem_desc(smem_u32(rqsnap), 16, 512, kSw64);
+  const uint64_t d_slot = smem_desc(smem_u32(slots), 16, 1024, kSw128);           // K-major
+  const uint64_t d_tile = smem_desc(smem_u32(slots), 16384, 1024, kSw128);        // MN-major
+  const uint64_t d_cq = smem_desc(smem_u32(smem + L::CQ), 8192, 512, kSw64);      // MN-major
+  constexpr uint32_t id_n64 = idesc_bf16(128, 64, false, false);
+  constexpr uint32_t id_n32 = idesc_bf16(128, 32, false, false);
+  constexpr uint32_t id_n16 = idesc_bf16(128, 16, false, false);
+  constexpr uint32_t id_ro = idesc_bf16(128, 64, false, true);     // slot x R' rows (MN-major)
+  constexpr uint32_t id_wo = idesc_bf16(128, 64, false, true);     // W~ (TMEM) x dout rows
+  constexpr uint32_t id_mq = idesc_bf16(128, 32, false, true);     // M (TMEM) x Q rows
+  constexpr uint32_t id_up = idesc_bf16(128, 64, true, true);
+  constexpr uint32_t id_rq = idesc_bf16(128, 32, true, true);
+
+  // ---- carry-in: R', Rq = the increments of segments g+1 .. G-1 (zero in
+  //      the increment kernel) ----
+  {
+    const float *seg0 = aggR + (size_t)bh * G * kAggFloats;
+    for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
+      const int mt = (!half && m == 2) ? 4 : m;
+      const int f = 128 * mt + r;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float acc[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+        if (!AGG && f < kD) {
+          for (int gp = g + 1; gp < G; ++gp) {
+            const float4 *src =
+                reinterpret_cast<const float4 *>(seg0 + (size_t)gp * kAggFloats + f * kDV + 16 * q4);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const float4 x = src[c4];
+              acc[4 * c4 + 0] += x.x;
+              acc[4 * c4 + 1] += x.y;
+              acc[4 * c4 + 2] += x.z;
+              acc[4 * c4 + 3] += x.w;
+            }
+          }
+        }
+        uint32_t bits[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) bits[c] = __float_as_uint(acc[c]);
+        tmem_st16(tbase + lane_off + kColR + 64 * mt + 16 * q4, bits);
+        if (!AGG && f < kD) {
+          *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4)) = pack8(bits);
+          *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4 + 1)) = pack8(bits + 8);
+        }
+      }
+    }
+    if (half) {
+      float acc[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+      if (!AGG && r < kDK) {
+        for (int gp = g + 1; gp < G; ++gp) {
+          const float4 *src =
+              reinterpret_cast<const float4 *>(seg0 + (size_t)gp * kAggFloats + kD * kDV + r * kDK);
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const float4 x = src[c4];
+            acc[4 * c4 + 0] += x.x;
+            acc[4 * c4 + 1] += x.y;
+            acc[4 * c4 + 2] += x.z;
+            acc[4 * c4 + 3] += x.w;
+          }
+        }
+      }
+      uint32_t bits[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) bits[c] = __float_as_uint(acc[c]);
+      tmem_st32(tbase + lane_off + kColRq, bits);
+      if (!AGG && quarter == 0) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(rqsnap + sw64(r, c)) = pack8(bits + 8 * c);
+      }
+    }
+  }
+
+  bool ok = true;
+  for (int i = 0; ok && i < nchunks; ++i) {
+    const int c0 = t0 + chunk_of(i) * kC;
+    const bool valid = c0 + r < T;
+    if (!(ok = wait_all(&bars[kBarLoadQ], i & 1))) break;
+    if (threadIdx.x < kC) {
+      const int t = c0 + threadIdx.x;
+      const bool vt = t < T;
+      invd_s[threadIdx.x] = vt ? 1.f / den[(size_t)bh * T + t] : 0.f;
+      c_s[threadIdx.x] = vt ? cvec[(size_t)bh * T + t] : 0.f;
+    }
+    __syncthreads();
+    if (!AGG) {
+      if (!(ok = wait_all(&bars[kBarLoadKV], i & 1))) break;
+      float kf[32];
+      row_f32(smem + L::K, r, kf);
+
+      // ---- dk carried: Y = V R'^T (J(k)^T contraction), U2 = K Rq ----
+      float h[32], g2R[32], kR[32];
+#pragma unroll
+      for (int l = 0; l < 32; ++l) {
+        h[l] = 0.f;
+        g2R[l] = 0.f;
+        kR[l] = kf[l];
+      }
+      if (half) rot<8>(kR);
+      float unused = 0.f;
+      for (int j = 0; ok && j < 5; ++j) {
+        ok = round([&] {
+          if (j == 0) {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ss(tbase + kColDk, adv(d_k, 32 * kk), adv(d_rq, 32 * kk), id_n32, kk);
+          }
+          if (j < 4) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + kColDv, adv(d_v, 32 * kk), adv(d_snap, 64 * j * 128 + 32 * kk), id_n64,
+                     kk);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + kColW, adv(d_v, 32 * kk), adv(d_snap, (256 + 64 * j) * 128 + 32 * kk),
+                     id_n64, kk);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + kColW, adv(d_v, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
+          }
+        });
+        if (!ok) break;
+        if (j == 0 && half == 0) {
+          uint32_t u[32];
+          tmem_ld32(tbase + lane_off + kColDk, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int l = 0; l < 32; l += 4)
+            *reinterpret_cast<float4 *>(ubuf + r * 32 + l) =
+                make_float4(__uint_as_float(u[l]), __uint_as_float(u[l + 1]),
+                            __uint_as_float(u[l + 2]), __uint_as_float(u[l + 3]));
+        }
+        if (j < 4) {
+          uint32_t x[32];
+          const uint32_t col = half ? kColW : kColDv;
+          tmem_ld32(tbase + lane_off + col, x);
+          tmem_wait_ld();
+          contract_offset<32>(x, kf, kR, h, g2R, unused);
+          tmem_ld32(tbase + lane_off + col + 32, x);
+          tmem_wait_ld();
+          contract_offset<32>(x, kf, kR, h, g2R, unused);
+        } else if (half) {
+          uint32_t x[16];
+          tmem_ld16(tbase + lane_off + kColW, x);
+          tmem_wait_ld();
+          contract_offset<16>(x, kf, kR, h, g2R, unused);
+        }
+      }
+      if (!ok) break;
+      if (half) {
+        rot<15>(g2R);
+      } else {
+        rot<24>(g2R);
+      }
+#pragma unroll
+      for (int l = 0; l < 32; ++l) h[l] += g2R[l];
+      if (half) {
+        float *row = xch + r * 36;
+#pragma unroll
+        for (int l = 0; l < 32; l += 4)
+          *reinterpret_cast<float4 *>(row + l) = make_float4(h[l], h[l + 1], h[l + 2], h[l + 3]);
+      }
+
+      // ---- dv carried: key products x R' rows, 64 features a slot, two slots a round ----
+      {
+        uint32_t XK[16], P[32], R[32];
+        load_pairs(smem + L::K, r, XK, P);
+#pragma unroll
+        for (int l = 0; l < 32; ++l) R[l] = P[l];
+        if (half) rotate_left(R, 8);
+        for (int j = 0; ok && j < 5; ++j) {
+          const int s9 = half ? 4 + j : j;
+          if (s9 <= 8 && (half || j < 4)) {
+            uint32_t w[32];
+            q_slot_words(P, R, s9 == kQSlotsPsd - 1, w);
+            uint8_t *slot = slots + 16384 * half;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+              *reinterpret_cast<uint4 *>(slot + sw128(r, cc)) =
+                  make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+            rotate_left(R, 2);
+          }
+          ok = round([&] {
+            const int sa = j, sb = 4 + j;
+            const int nk_b = sb == kQSlotsPsd - 1 ? 1 : 4;
+            if (j < 4) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tbase + kColDv, adv(d_slot, 32 * kk), adv(d_snap_mn, (64 * sa + 16 * kk) * 128),
+                       id_ro, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            for (int kk = 0; kk < nk_b; ++kk)
+              mma_ss(tbase + kColDv, adv(d_slot, 16384 + 32 * kk),
+                     adv(d_snap_mn, (64 * sb + 16 * kk) * 128), id_ro, 1u);
+          });
+        }
+        if (!ok) break;
+      }
+
+      // ---- intra-chunk: four quarters of 32 queries t >= s ----
+      const uint32_t ws_col = kColW + 8 * half;           // this half's W~ words
+      const uint32_t ms_col = kColW + 16 + 8 * half;      // this half's M words
+      for (int qt = 0; ok && qt < 4; ++qt) {
+        ok = round([&] {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_ss(tbase + kColW, adv(d_k, 32 * kk), adv(d_q, 2048 * qt + 32 * kk), id_n32, kk);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tbase + kColW + 32, adv(d_v, 32 * kk), adv(d_o, 4096 * qt + 32 * kk), id_n32, kk);
+        });
+        if (!ok) break;
+        uint32_t a[16], dp[16], wv[8], mv[8];
+        tmem_ld16(tbase + lane_off + kColW + 16 * half, a);
+        tmem_ld16(tbase + lane_off + kColW + 32 + 16 * half, dp);
+        tmem_wait_ld();
+        const int tb = 32 * qt + 16 * half;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float wq[2], mq[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int t = tb + 2 * j + e;
+            const float av = __uint_as_float(a[2 * j + e]);
+            const float it = invd_s[t], ct = c_s[t];
+            const bool keep = t >= r;
+            wq[e] = keep ? av * av * it : 0.f;
+            mq[e] = keep ? 2.f * av * fmaf(__uint_as_float(dp[2 * j + e]), it, ct) : 0.f;
+          }
+          wv[j] = pack_bf16x2(wq[0], wq[1]);
+          mv[j] = pack_bf16x2(mq[0], mq[1]);
+        }
+        __syncthreads();        // every thread has read its columns before W~, M overwrite them
+        tmem_st8(tbase + lane_off + ws_col, wv);
+        tmem_st8(tbase + lane_off + ms_col, mv);
+        ok = round([&] {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_ts(tbase + kColDv, tbase + kColW + 8 * kk, adv(d_o_mn, 4096 * qt + 2048 * kk), id_wo, 1u);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk)
+            mma_ts(tbase + kColDk, tbase + kColW + 16 + 8 * kk, adv(d_q_mn, 2048 * qt + 1024 * kk), id_mq,
+                   (qt > 0 || kk > 0) ? 1u : 0u);
+        });
+      }
+      if (!ok) break;
+      if (threadIdx.x == 0 && i + 1 < nchunks) load_kv(i + 1);    // K, V no longer read
+      // ---- outputs: dk = intra + J(k)^T Y + 2 Rq k (half 0), dv (half 1) ----
+      if (!half) {
+        uint32_t acc[32];
+        tmem_ld32(tbase + lane_off + kColDk, acc);
+        tmem_wait_ld();
+        const float *row = xch + r * 36, *u = ubuf + r * 32;
+        if (valid) {
+          uint4 *dst = reinterpret_cast<uint4 *>(dk + ((size_t)bh * T + c0 + r) * kDK);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j2 = 0; j2 < 4; ++j2) {
+              const int l0 = 8 * c + 2 * j2;
+              w[j2] = pack_bf16x2(__uint_as_float(acc[l0]) + h[l0] + row[l0] + 2.f * u[l0],
+                                  __uint_as_float(acc[l0 + 1]) + h[l0 + 1] + row[l0 + 1] + 2.f * u[l0 + 1]);
+            }
+            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      } else {
+        uint32_t acc[32];
+#pragma unroll 1
+        for (int hv = 0; hv < 2; ++hv) {
+          tmem_ld32(tbase + lane_off + kColDv + 32 * hv, acc);
+          tmem_wait_ld();
+          if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(dv + ((size_t)bh * T + c0 + r) * kDV + 32 * hv);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dst[c] = pack8(acc + 8 * c);
+          }
+        }
+      }
+    }
+    if (!AGG && i == nchunks - 1) break;       // the state before the segment is not needed
+
+    // ---- update: R' += (m p(q) / d)^T dout (tiles (0, 2), (1, 3), (4)), Rq += Q^T diag(c) Q ----
+    {
+      uint32_t XQ[16], P[32], R2[32];
+      load_pairs(smem + L::Q, r, XQ, P);
+      const float inv_r = invd_s[r], c_r = c_s[r];
+      const uint32_t two_inv = pack_bf16x2(2.f * inv_r, 2.f * inv_r);
+#pragma unroll
+      for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[l], two_inv);   // x 2 / d_t
+      if (half) {
+        rotate_left(R2, 8);
+      } else {
+        // c_t q_t as bf16, the Rq update's A operand
+        const uint32_t cc2 = pack_bf16x2(c_r, c_r);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 x = *reinterpret_cast<const uint4 *>(smem + L::Q + sw64(r, c));
+          *reinterpret_cast<uint4 *>(smem + L::CQ + sw64(r, c)) =
+              make_uint4(bmul2(x.x, cc2), bmul2(x.y, cc2), bmul2(x.z, cc2), bmul2(x.w, cc2));
+        }
+      }
+      for (int u = 0; ok && u < 3; ++u) {
+        const int m = half ? (u < 2 ? 2 + u : -1) : (u < 2 ? u : 4);
+        if (m >= 0)
+          write_tile(slots + 32768 * half, r, m == kTiles - 1, m == 0 ? 0x3f003f00u : 0x3f803f80u,
+                     P, R2);
+        if (!half && u == 1) {
+          rotate_left(R2, 12);
+        } else {
+          rotate_left(R2, 4);
+        }
+        ok = round([&] {
+          const int ma = u < 2 ? u : 4, mb = 2 + u;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tbase + kColR + 64 * ma, adv(d_tile, 2048 * kk), adv(d_o_mn, 2048 * kk), id_up, 1);
+          if (u < 2) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + kColR + 64 * mb, adv(d_tile, 32768 + 2048 * kk), adv(d_o_mn, 2048 * kk),
+                     id_up, 1);
+          }
+          if (u == 0) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + kColRq, adv(d_cq, 1024 * kk), adv(d_q_mn, 1024 * kk), id_rq, 1);
+          }
+        });
+      }
+      if (!ok) break;
+      if (threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);     // Q, dout no longer read
+    }
+    // ---- snapshot R' (half 0: tiles 0, 1, 4; half 1: tiles 2, 3) and Rq ----
+    if constexpr (!AGG) {
+    for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
+      const int mt = (!half && m == 2) ? 4 : m;
+      if (mt == 4 && quarter != 0) continue;
+      const int f = 128 * mt + r;
+      uint32_t a[32], b2[32];
+      tmem_ld32(tbase + lane_off + kColR + 64 * mt, a);
+      tmem_ld32(tbase + lane_off + kColR + 64 * mt + 32, b2);
+      tmem_wait_ld();
+      if (f < kD) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          *reinterpret_cast<uint4 *>(snap + sw128(f, q4)) = pack8(a + 8 * q4);
+          *reinterpret_cast<uint4 *>(snap + sw128(f, 4 + q4)) = pack8(b2 + 8 * q4);
+        }
+      }
+    }
+    if (half && quarter == 0) {
+      uint32_t zr[32];
+      tmem_ld32(tbase + lane_off + kColRq, zr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(rqsnap + sw64(r, c)) = pack8(zr + 8 * c);
+    }
+    }
+  }
+
+  // ---- the increment kernel writes its segment's (R', Rq) ----
+  if (AGG && ok && nchunks > 0) {
+    float *dst = aggR + ((size_t)bh * G + g) * kAggFloats;
+    for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
+      const int mt = (!half && m == 2) ? 4 : m;
+      if (mt == 4 && quarter != 0) continue;
+      const int f = 128 * mt + r;
+      uint32_t a[32], b2[32];
+      tmem_ld32(tbase + lane_off + kColR + 64 * mt, a);
+      tmem_ld32(tbase + lane_off + kColR + 64 * mt + 32, b2);
+      tmem_wait_ld();
+      if (f < kD) {
+        float4 *row = reinterpret_cast<float4 *>(dst + (size_t)f * kDV);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          row[c] = make_float4(__uint_as_float(a[4 * c]), __uint_as_float(a[4 * c + 1]),
+                               __uint_as_float(a[4 * c + 2]), __uint_as_float(a[4 * c + 3]));
+          row[8 + c] = make_float4(__uint_as_float(b2[4 * c]), __uint_as_float(b2[4 * c + 1]),
+                                   __uint_as_float(b2[4 * c + 2]), __uint_as_float(b2[4 * c + 3]));
+        }
+      }
+    }
+    if (half && quarter == 0) {
+      uint32_t zr[32];
+      tmem_ld32(tbase + lane_off + kColRq, zr);
+      tmem_wait_ld();
+      float4 *row = reinterpret_cast<float4 *>(dst + kD * kDV + r * kDK);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        row[c] = make_float4(__uint_as_float(zr[4 * c]), __uint_as_float(zr[4 * c + 1]),
+                             __uint_as_float(zr[4 * c + 2]), __uint_as_float(zr[4 * c + 3]));
+    }
+  }
+  if (*abort_flag && threadIdx.x == 0) flag_status(status, kStatusDeviceTimeout);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tbase, kTmemCols);
+}
+
 }  // namespace
 
 cudaError_t tc_bwd_dq(const BackwardLaunch &a, float *aggS, int G, int seg_len) {
@@ -573,6 +1135,34 @@ cudaError_t tc_bwd_dq(const BackwardLaunch &a, float *aggS, int G, int seg_len) 
   bwd_dq_tc_kernel<<<(unsigned)(a.BH * G), kBThreads, DqSmem::Bytes, a.stream>>>(
       tq, tk, tv, to, aggS, static_cast<__nv_bfloat16 *>(a.dq), a.den, a.c, a.status, a.T, G,
       seg_len);
+  return cudaGetLastError();
+}
+
+
+cudaError_t tc_bwd_dkdv(const BackwardLaunch &a, float *aggR, int G, int seg_len) {
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tma_3d_bf16(&tq, a.q, kDK, a.T, a.BH, kC) ||
+      !make_tma_3d_bf16(&tk, a.k, kDK, a.T, a.BH, kC) ||
+      !make_tma_3d_bf16(&tv, a.v, kDV, a.T, a.BH, kC) ||
+      !make_tma_3d_bf16(&to, a.dout, kDV, a.T, a.BH, kC))
+    return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (G > 1) {
+    auto kinc = bwd_dkdv_tc_kernel<true>;
+    e = cudaFuncSetAttribute(kinc, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvSmem::Bytes);
+    if (e != cudaSuccess) return e;
+    ProfileScope prof("tc_bwd_suffix_increment", a.stream);
+    kinc<<<(unsigned)(a.BH * (G - 1)), kBThreads, DkvSmem::Bytes, a.stream>>>(
+        tq, tk, tv, to, aggR, a.den, a.c, nullptr, nullptr, a.status, a.T, G, seg_len);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  auto kern = bwd_dkdv_tc_kernel<false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvSmem::Bytes);
+  if (e != cudaSuccess) return e;
+  ProfileScope prof("tc_bwd_dkdv", a.stream);
+  kern<<<(unsigned)(a.BH * G), kBThreads, DkvSmem::Bytes, a.stream>>>(
+      tq, tk, tv, to, aggR, a.den, a.c, static_cast<__nv_bfloat16 *>(a.dk),
+      static_cast<__nv_bfloat16 *>(a.dv), a.status, a.T, G, seg_len);
   return cudaGetLastError();
 }
 

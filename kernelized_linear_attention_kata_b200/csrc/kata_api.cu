@@ -197,14 +197,14 @@ struct BackwardRun {
   static constexpr bool kBaseFeaturesOnly = true;     // the gradient covers PSD and first-order
   kata_dtype_t dtype;
   BackwardLaunch a;
-  bool tc;                 // bf16 PSD d_k = 32, d_v = 64: the tensor-core dq pass
+  bool tc;                 // bf16 PSD d_k = 32, d_v = 64: the tensor-core kernels
   int tc_G, tc_seg_len;
   template <int DK, int DV, int FEAT> kata_status_t operator()() {
     cudaError_t e;
     if constexpr (DK == 32 && DV == 64 && FEAT == kPSD) {
       if (tc) {
         e = tc_bwd_dq(a, a.aggS, tc_G, tc_seg_len);
-        if (e == cudaSuccess) e = simt_backward_dkdv<DK, DV, FEAT, __nv_bfloat16>(a);
+        if (e == cudaSuccess) e = tc_bwd_dkdv(a, a.aggR, tc_G, tc_seg_len);
         return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
       }
     }

@@ -111,6 +111,10 @@ size_t tc_chunked_agg_floats();   // floats of one segment increment
 // aggS (PSD tensor-core layout, G per head), then dq and, per token, d_t and
 // c_t (a.den, a.c) for the suffix pass; G segments of seg_len tokens.
 cudaError_t tc_bwd_dq(const BackwardLaunch &a, float *aggS, int G, int seg_len);
+// Tensor-core gradients with respect to k and v (same shapes), from a.den and
+// a.c of the dq pass: the suffix increments of segments 1 .. G-1 into aggR
+// (same layout), then each segment's chunks in reverse order.
+cudaError_t tc_bwd_dkdv(const BackwardLaunch &a, float *aggR, int G, int seg_len);
 // Segment increments of the PSD tensor-core layout (d_k = 32, d_v = 64 bf16):
 // segments 0 .. G_inc - 1 of G_total (seg_len tokens each, whole 128-token
 // chunks) into agg[bh][g], G_total increments per head.

@@ -63,6 +63,10 @@ CASES = [
     ("psd", "bf16", 1, 2, 300, 32, 64, 128),
     ("psd", "bf16", 2, 2, 129, 16, 64, 64),
     ("psd", "bf16", 2, 80, 70, 32, 64, 64),
+    # the tensor-core kernels (bf16, d_k = 32, d_v = 64): one-chunk segments
+    # with a ragged last chunk, and segments of several chunks
+    ("psd", "bf16", 1, 3, 1000, 32, 64, 128),
+    ("psd", "bf16", 2, 20, 2000, 32, 64, 128),
     ("first_order", "f32", 1, 1, 1, 64, 64, 64),
     ("first_order", "f32", 1, 2, 191, 64, 64, 64),
     ("first_order", "f32", 2, 2, 100, 16, 32, 32),
@@ -134,7 +138,12 @@ def test_backward_long_workload_sampled_rows():
     w = W.LONG
     (q, k, v, dy), (dq, dk, dv) = run_gpu(w)
     rng = np.random.default_rng(17)
-    rows = np.array(sorted(set([0, 1, 127, 128, 4095, w.T // 2, w.T - 2, w.T - 1])
+    # segment starts of the tensor-core split (9 segments of 114 chunks per
+    # head on 148 SMs) and the rows just before them, where the carried
+    # prefix and suffix states change hands
+    seg = 114 * 128
+    bounds = set(x for gi in range(1, 9) for x in (gi * seg - 1, gi * seg))
+    rows = np.array(sorted(set([0, 1, 127, 128, 4095, w.T // 2, w.T - 2, w.T - 1]) | bounds
                            | set(int(x) for x in rng.integers(0, w.T, size=24))))
     for h in (0, w.H - 1):
         ref = O.backward_rows(f64(q)[0, h], f64(k)[0, h], f64(v)[0, h], f64(dy)[0, h], rows, w.feature)
