@@ -137,6 +137,9 @@ KERNEL_SOURCES = {
     "tc_quadratic": ["quadratic_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_fo_pass": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_fo_increment": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
+    "tc_bwd_dq": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
+    "tc_bwd_dkdv": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
+    "tc_bwd_suffix_increment": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
 }
 
 
