@@ -345,8 +345,12 @@ KATA_API size_t kata_bwd_chunked_workspace_bytes(int B, int H, int T, int d_k, i
  *                      256-byte aligned, contents on entry ignored; holds the
  *                      status word afterwards (kata_workspace_status reports
  *                      a non-positive normaliser as for the forward).
- * Arithmetic is fp32 (CUDA cores) for both dtypes. Returns KATA_OK when the
- * work was launched; B, H or T = 0 launches nothing.
+ * bf16 PSD with d_k = 32, d_v = 64, C in {64, 128} and 16-byte aligned
+ * pointers runs on the tensor cores (bf16 MMA operands: the inputs, the
+ * state snapshots and the intra-chunk gradient blocks; fp32 accumulation;
+ * the same bf16 tolerance as the forward). Every other case computes in
+ * fp32 on the CUDA cores. Returns KATA_OK when the work was launched; B, H
+ * or T = 0 launches nothing.
  */
 KATA_API kata_status_t kata_bwd_chunked(const void *q, const void *k, const void *v,
                                         const void *dout, void *dq, void *dk, void *dv,
