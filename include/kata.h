@@ -118,8 +118,13 @@ typedef enum {
     KATA_PATH_TENSOR_CORE_FIRST_ORDER = 2, /* tcgen05/TMEM kernels, bf16
                                        first-order, d_k = d_v = 64,
                                        C in {64, 128}                          */
-    KATA_PATH_CUDA_CORE = 3         /* fp32 FFMA kernels: the fp32 path and
+    KATA_PATH_CUDA_CORE = 3,        /* fp32 FFMA kernels: the fp32 path and
                                        every other supported shape            */
+    KATA_PATH_TENSOR_CORE_MULTI_FACTOR = 4 /* tcgen05/TMEM kernels, bf16
+                                       MULTI_PSD2 / SUMMED_PSD2, d_k = 32,
+                                       d_v = 64, C in {64, 128} (the
+                                       state-only call kata_chunked_state
+                                       runs them on the CUDA cores)           */
 } kata_path_t;
 
 /* How kata_fwd_chunked will run a problem (see kata_fwd_chunked_plan). */

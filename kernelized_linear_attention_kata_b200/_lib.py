@@ -26,9 +26,11 @@ KATA_PATH_NONE = 0
 KATA_PATH_TENSOR_CORE_PSD = 1
 KATA_PATH_TENSOR_CORE_FIRST_ORDER = 2
 KATA_PATH_CUDA_CORE = 3
+KATA_PATH_TENSOR_CORE_MULTI_FACTOR = 4
 PATH_NAMES = {KATA_PATH_NONE: "none", KATA_PATH_TENSOR_CORE_PSD: "tensor_core_psd",
               KATA_PATH_TENSOR_CORE_FIRST_ORDER: "tensor_core_first_order",
-              KATA_PATH_CUDA_CORE: "cuda_core"}
+              KATA_PATH_CUDA_CORE: "cuda_core",
+              KATA_PATH_TENSOR_CORE_MULTI_FACTOR: "tensor_core_multi_factor"}
 
 KATA_DTYPE_F32 = 0
 KATA_DTYPE_BF16 = 1

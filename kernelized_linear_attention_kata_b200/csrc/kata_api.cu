@@ -75,6 +75,11 @@ size_t increments_per_head(kata_path_t path, long long BH, int T, int sms, bool 
     tc_chunked_layout(BH, T, sms, sequential, &G, &seg_len, &P);
     return (size_t)G * (size_t)P;
   }
+  if (path == KATA_PATH_TENSOR_CORE_MULTI_FACTOR) {
+    int G, seg_len;
+    var_tc_layout(BH, T, sms, sequential, &G, &seg_len);
+    return (size_t)G;
+  }
   return (size_t)sp.G;
 }
 
@@ -159,6 +164,8 @@ kata_path_t chunked_path(const ChunkedLaunch &a, int d_k, int d_v, int C, kata_d
     return KATA_PATH_TENSOR_CORE_PSD;
   if (dtype == KATA_DTYPE_BF16 && fo_tc_supported(a, d_k, d_v, C, feature))
     return KATA_PATH_TENSOR_CORE_FIRST_ORDER;
+  if (dtype == KATA_DTYPE_BF16 && var_tc_supported(a, d_k, d_v, C, feature))
+    return KATA_PATH_TENSOR_CORE_MULTI_FACTOR;
   return KATA_PATH_CUDA_CORE;
 }
 
@@ -171,6 +178,7 @@ struct ChunkedRun {
     switch (chunked_path(a, DK, DV, a.C, dtype, FEAT)) {
       case KATA_PATH_TENSOR_CORE_PSD: e = tc_chunked(a); break;
       case KATA_PATH_TENSOR_CORE_FIRST_ORDER: e = fo_tc(a); break;
+      case KATA_PATH_TENSOR_CORE_MULTI_FACTOR: e = var_tc(a, FEAT); break;
       default:
         e = dtype == KATA_DTYPE_F32 ? simt_chunked<DK, DV, FEAT, float>(a)
                                     : simt_chunked<DK, DV, FEAT, __nv_bfloat16>(a);
@@ -325,6 +333,9 @@ kata_status_t kata_fwd_chunked_plan(int B, int H, int T, int d_k, int d_v, int C
   } else if (p.path == KATA_PATH_TENSOR_CORE_FIRST_ORDER) {
     p.chunk_tokens = 128;
     tile_segments(T, 128, sp.G, &p.segments, &p.segment_tokens);
+  } else if (p.path == KATA_PATH_TENSOR_CORE_MULTI_FACTOR) {
+    p.chunk_tokens = 128;
+    var_tc_layout(BH, T, sms, sequential != 0, &p.segments, &p.segment_tokens);
   } else {
     p.chunk_tokens = C;
     p.segments = sp.G;
@@ -348,8 +359,11 @@ size_t kata_fwd_chunked_workspace_bytes(int B, int H, int T, int d_k, int d_v, i
   ChunkedLaunch a{aligned, aligned, aligned, aligned, BH, T, C, nullptr, nullptr, nullptr,
                   nullptr, sp.G, sp.seg_len, nullptr};
   const kata_path_t path = chunked_path(a, d_k, d_v, C, dtype, feature);
-  return workspace_bytes_for(BH, (int)kata_state_dim(d_k, feature), d_k, d_v,
-                             increments_per_head(path, BH, T, sms, false, sp));
+  size_t incs = increments_per_head(path, BH, T, sms, false, sp);
+  // the variants' state-only call (kata_chunked_state) runs on the CUDA cores
+  // with their split: the size covers both
+  if (path == KATA_PATH_TENSOR_CORE_MULTI_FACTOR && (size_t)sp.G > incs) incs = (size_t)sp.G;
+  return workspace_bytes_for(BH, (int)kata_state_dim(d_k, feature), d_k, d_v, incs);
 }
 
 kata_status_t kata_fwd_chunked(const void *q, const void *k, const void *v, void *o, int B, int H,

@@ -106,6 +106,12 @@ cudaError_t tc_quadratic(const QuadraticLaunch &a, int d_k, int d_v, int feature
 bool tc_chunked_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
 cudaError_t tc_chunked(const ChunkedLaunch &a);
 size_t tc_chunked_agg_floats();   // floats of one segment increment
+// Tensor-core chunked forward of the two-factor variants (kMg2, kSg2; bf16,
+// d_k = 32, d_v = 64, C in {64, 128}; not the state-only call): G segments
+// of seg_len tokens (whole 128-token chunks), one increment per segment.
+bool var_tc_supported(const ChunkedLaunch &a, int d_k, int d_v, int C, int feature);
+void var_tc_layout(long long BH, int T, int sms, bool sequential, int *G, int *seg_len);
+cudaError_t var_tc(const ChunkedLaunch &a, int feature);
 // Tensor-core gradient with respect to q of the PSD chunked forward (bf16,
 // d_k = 32, d_v = 64): the forward's increments of segments 0 .. G-2 into
 // aggS (PSD tensor-core layout, G per head), then dq and, per token, d_t and

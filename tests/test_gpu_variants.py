@@ -145,3 +145,57 @@ def test_variant_backward_is_rejected():
     v = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(Exception):
         api.bwd_chunked(q, q, v, v, 64, "mg2")
+
+
+@pytest.mark.parametrize("feature", sorted(VARIANTS))
+def test_variant_kernel_family(feature):
+    """bf16 with d_k = 32, d_v = 64 and C in {64, 128} runs on the tensor
+    cores; fp32, other chunk sizes and other shapes on the CUDA cores."""
+    def path(dtype, d_k, d_v, C):
+        return api.fwd_chunked_plan(1, 16, 131072, d_k, d_v, C, dtype, feature)["path"]
+    assert path(torch.bfloat16, 32, 64, 128) == "tensor_core_multi_factor"
+    assert path(torch.bfloat16, 32, 64, 64) == "tensor_core_multi_factor"
+    assert path(torch.float32, 32, 64, 128) == "cuda_core"
+    assert path(torch.bfloat16, 32, 64, 32) == "cuda_core"
+    assert path(torch.bfloat16, 16, 16, 64) == "cuda_core"
+
+
+@pytest.mark.parametrize("feature", sorted(VARIANTS))
+def test_variant_tc_state_and_continuation(feature):
+    """The tensor-core path's returned state, element by element, and a
+    sequence processed in two calls (the second from the first's state)
+    against the definition on the whole sequence.
+
+    State bound per entry: fp32 accumulation of T terms, (T + 8) 2^-23
+    sum_t |a_t|, plus one bf16 rounding (unit roundoff 2^-8) of each key
+    feature entering the update MMA, at most 2^-8 sum_t |a_t|; z is formed
+    from exact products (Z = K^T K) and gets the accumulation term only."""
+    variant = VARIANTS[feature]
+    B, H, T, T1, d_k, d_v = 1, 3, 700, 300, 32, 64
+    q, k, v = inputs(B, H, T, d_k, d_v, "bf16", seed=131)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    y, S, z = api.fwd_chunked(qd, kd, vd, 128, feature, return_state=True)
+    ref = oracle(V.forward_variant_brute_force, q, k, v, variant, 2)
+    assert rel_err(y.float().cpu().numpy(), ref) <= TOL["bf16"]
+    qn, kn, vn = f64(q), f64(k), f64(v)
+    for h in range(H):
+        _, S_ref, z_ref = V.forward_variant_recurrent(qn[0, h], kn[0, h], vn[0, h], variant, 2,
+                                                      return_state=True)
+        _, S_abs, z_abs = V.forward_variant_recurrent(qn[0, h], np.abs(kn[0, h]), np.abs(vn[0, h]),
+                                                      variant, 2, return_state=True)
+        acc = (T + 8) * 2.0 ** -23
+        assert np.all(np.abs(S[0, h].cpu().numpy() - S_ref) <= (acc + 2.0 ** -8) * S_abs + 1e-30), h
+        assert np.all(np.abs(z[0, h].cpu().numpy() - z_ref) <= acc * z_abs + 1e-30), h
+    # two calls: tokens [0, T1), then [T1, T) from the first call's state
+    y1, S1, z1 = api.fwd_chunked(qd[:, :, :T1].contiguous(), kd[:, :, :T1].contiguous(),
+                                 vd[:, :, :T1].contiguous(), 128, feature, return_state=True)
+    y2 = torch.empty_like(vd[:, :, T1:])
+    S2 = torch.empty_like(S)
+    z2 = torch.empty_like(z)
+    api.kata_fwd_chunked(qd[:, :, T1:].contiguous(), kd[:, :, T1:].contiguous(),
+                         vd[:, :, T1:].contiguous(), y2, 64, feature, S_out=S2, z_out=z2,
+                         S0=S1, z0=z1)
+    yy = torch.cat([y1, y2], dim=2).float().cpu().numpy()
+    assert rel_err(yy, ref) <= TOL["bf16"]
+    assert torch.allclose(S2, S, rtol=1e-3, atol=1e-3 * float(S.abs().max()))
+    assert torch.allclose(z2, z, rtol=1e-5, atol=1e-5 * float(z.abs().max()))
