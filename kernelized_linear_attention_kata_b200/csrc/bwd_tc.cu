@@ -106,14 +106,15 @@ __device__ __forceinline__ void rot(float (&R)[32]) {
 // for l < nl) with its X values: x[l] = X_(d,l) (the state's doubled rows make
 // X_f = m_f (S dout)_f). qR = q rotated by d, g2R accumulates the Jacobian's
 // second term in the same rotated frame; both are rotated by one afterwards.
-template <int NL>
+// DN adds the contraction with the features themselves (dout . n).
+template <int NL, bool DN = true>
 __device__ __forceinline__ void contract_offset(const uint32_t *x, const float (&q)[32],
                                                 float (&qR)[32], float (&h)[32], float (&g2R)[32],
                                                 float &dn) {
 #pragma unroll
   for (int l = 0; l < NL; ++l) {
     const float xv = __uint_as_float(x[l]);
-    dn = fmaf(q[l] * qR[l], xv, dn);
+    if constexpr (DN) dn = fmaf(q[l] * qR[l], xv, dn);
     h[l] = fmaf(qR[l], xv, h[l]);
     g2R[l] = fmaf(q[l], xv, g2R[l]);
   }
@@ -852,15 +853,15 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
           const uint32_t col = half ? kColW : kColDv;
           tmem_ld32(tbase + lane_off + col, x);
           tmem_wait_ld();
-          contract_offset<32>(x, kf, kR, h, g2R, unused);
+          contract_offset<32, false>(x, kf, kR, h, g2R, unused);
           tmem_ld32(tbase + lane_off + col + 32, x);
           tmem_wait_ld();
-          contract_offset<32>(x, kf, kR, h, g2R, unused);
+          contract_offset<32, false>(x, kf, kR, h, g2R, unused);
         } else if (half) {
           uint32_t x[16];
           tmem_ld16(tbase + lane_off + kColW, x);
           tmem_wait_ld();
-          contract_offset<16>(x, kf, kR, h, g2R, unused);
+          contract_offset<16, false>(x, kf, kR, h, g2R, unused);
         }
       }
       if (!ok) break;
