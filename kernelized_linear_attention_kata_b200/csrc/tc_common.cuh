@@ -296,75 +296,6 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 }
 
 // ---------------------------------------------------------------------------
-// Thread-block clusters (distributed shared memory between the CTAs of a
-// cluster on this GPU; no multicast anywhere)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-// Address, in the shared::cluster window, of the same shared-memory offset in
-// CTA `rank` of this cluster.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-
-// Arrives on an mbarrier of another CTA of the cluster (address from
-// mapa_shared), releasing this thread's earlier writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait on a local mbarrier whose phase is completed by another CTA of
-// the cluster (acquire at cluster scope); same limit and abort rule as mbar_wait.
-static __device__ __noinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
-                                                      volatile int *abort) {
-  if (mbar_try_wait_cluster(bar, parity, 0u)) return true;
-  const uint64_t start = global_ns();
-  for (;;) {
-    if (mbar_try_wait_cluster(bar, parity, kSuspendHintNs)) return true;
-    if (*abort) return false;
-    if (global_ns() - start > kWaitLimitNs) {
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
-// All threads of every CTA of the cluster (aligned: every thread of each warp).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-
-// ---------------------------------------------------------------------------
 // Packing
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
