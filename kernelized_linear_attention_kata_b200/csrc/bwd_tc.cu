@@ -879,16 +879,19 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
           *reinterpret_cast<float4 *>(row + l) = make_float4(h[l], h[l + 1], h[l + 2], h[l + 3]);
       }
 
-      // ---- dv carried: key products x R' rows, 64 features a slot, two slots a round ----
+      // ---- dv carried (key products x R' rows, 64 features a slot, half 0
+      //      slots 0..3, half 1 slots 4..8, one pair a round) interleaved with
+      //      the intra-chunk quarters of 32 queries t >= s ----
       {
         uint32_t XK[16], P[32], R[32];
         load_pairs(smem + L::K, r, XK, P);
 #pragma unroll
         for (int l = 0; l < 32; ++l) R[l] = P[l];
         if (half) rotate_left(R, 8);
-        for (int j = 0; ok && j < 5; ++j) {
-          const int s9 = half ? 4 + j : j;
-          if (s9 <= 8 && (half || j < 4)) {
+        // slot pair j: half 0 writes slot j (j < 4), half 1 slot 4 + j
+        auto write_slot = [&](int j) {
+          if (half || j < 4) {
+            const int s9 = half ? 4 + j : j;
             uint32_t w[32];
             q_slot_words(P, R, s9 == kQSlotsPsd - 1, w);
             uint8_t *slot = slots + 16384 * half;
@@ -898,68 +901,70 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                   make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
             rotate_left(R, 2);
           }
-          ok = round([&] {
-            const int sa = j, sb = 4 + j;
-            const int nk_b = sb == kQSlotsPsd - 1 ? 1 : 4;
-            if (j < 4) {
+        };
+        auto issue_slots = [&](int j) {
+          const int sa = j, sb = 4 + j;
+          const int nk_b = sb == kQSlotsPsd - 1 ? 1 : 4;
+          if (j < 4) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tbase + kColDv, adv(d_slot, 32 * kk), adv(d_snap_mn, (64 * sa + 16 * kk) * 128),
-                       id_ro, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + kColDv, adv(d_slot, 32 * kk), adv(d_snap_mn, (64 * sa + 16 * kk) * 128),
+                     id_ro, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          for (int kk = 0; kk < nk_b; ++kk)
+            mma_ss(tbase + kColDv, adv(d_slot, 16384 + 32 * kk),
+                   adv(d_snap_mn, (64 * sb + 16 * kk) * 128), id_ro, 1u);
+        };
+        write_slot(0);
+        const uint32_t ws_col = kColW + 8 * half;           // this half's W~ words
+        const uint32_t ms_col = kColW + 16 + 8 * half;      // this half's M words
+        for (int qt = 0; ok && qt < 4; ++qt) {
+          ok = round([&] {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ss(tbase + kColW, adv(d_k, 32 * kk), adv(d_q, 2048 * qt + 32 * kk), id_n32, kk);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + kColW + 32, adv(d_v, 32 * kk), adv(d_o, 4096 * qt + 32 * kk), id_n32, kk);
+            issue_slots(qt);
+          });
+          if (!ok) break;
+          uint32_t a[16], dp[16], wv[8], mv[8];
+          tmem_ld16(tbase + lane_off + kColW + 16 * half, a);
+          tmem_ld16(tbase + lane_off + kColW + 32 + 16 * half, dp);
+          tmem_wait_ld();
+          const int tb = 32 * qt + 16 * half;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float wq[2], mq[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int t = tb + 2 * j + e;
+              const float av = __uint_as_float(a[2 * j + e]);
+              const float it = invd_s[t], ct = c_s[t];
+              const bool keep = t >= r;
+              wq[e] = keep ? av * av * it : 0.f;
+              mq[e] = keep ? 2.f * av * fmaf(__uint_as_float(dp[2 * j + e]), it, ct) : 0.f;
             }
-            for (int kk = 0; kk < nk_b; ++kk)
-              mma_ss(tbase + kColDv, adv(d_slot, 16384 + 32 * kk),
-                     adv(d_snap_mn, (64 * sb + 16 * kk) * 128), id_ro, 1u);
+            wv[j] = pack_bf16x2(wq[0], wq[1]);
+            mv[j] = pack_bf16x2(mq[0], mq[1]);
+          }
+          __syncthreads();        // every thread has read its columns before W~, M overwrite them
+          tmem_st8(tbase + lane_off + ws_col, wv);
+          tmem_st8(tbase + lane_off + ms_col, mv);
+          write_slot(qt + 1);     // the previous pair's slots were read by the last round
+          ok = round([&] {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ts(tbase + kColDv, tbase + kColW + 8 * kk, adv(d_o_mn, 4096 * qt + 2048 * kk), id_wo,
+                     1u);
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ts(tbase + kColDk, tbase + kColW + 16 + 8 * kk, adv(d_q_mn, 2048 * qt + 1024 * kk),
+                     id_mq, (qt > 0 || kk > 0) ? 1u : 0u);
+            if (qt == 3) issue_slots(4);
           });
         }
-        if (!ok) break;
-      }
-
-      // ---- intra-chunk: four quarters of 32 queries t >= s ----
-      const uint32_t ws_col = kColW + 8 * half;           // this half's W~ words
-      const uint32_t ms_col = kColW + 16 + 8 * half;      // this half's M words
-      for (int qt = 0; ok && qt < 4; ++qt) {
-        ok = round([&] {
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_ss(tbase + kColW, adv(d_k, 32 * kk), adv(d_q, 2048 * qt + 32 * kk), id_n32, kk);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tbase + kColW + 32, adv(d_v, 32 * kk), adv(d_o, 4096 * qt + 32 * kk), id_n32, kk);
-        });
-        if (!ok) break;
-        uint32_t a[16], dp[16], wv[8], mv[8];
-        tmem_ld16(tbase + lane_off + kColW + 16 * half, a);
-        tmem_ld16(tbase + lane_off + kColW + 32 + 16 * half, dp);
-        tmem_wait_ld();
-        const int tb = 32 * qt + 16 * half;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float wq[2], mq[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int t = tb + 2 * j + e;
-            const float av = __uint_as_float(a[2 * j + e]);
-            const float it = invd_s[t], ct = c_s[t];
-            const bool keep = t >= r;
-            wq[e] = keep ? av * av * it : 0.f;
-            mq[e] = keep ? 2.f * av * fmaf(__uint_as_float(dp[2 * j + e]), it, ct) : 0.f;
-          }
-          wv[j] = pack_bf16x2(wq[0], wq[1]);
-          mv[j] = pack_bf16x2(mq[0], mq[1]);
-        }
-        __syncthreads();        // every thread has read its columns before W~, M overwrite them
-        tmem_st8(tbase + lane_off + ws_col, wv);
-        tmem_st8(tbase + lane_off + ms_col, mv);
-        ok = round([&] {
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_ts(tbase + kColDv, tbase + kColW + 8 * kk, adv(d_o_mn, 4096 * qt + 2048 * kk), id_wo, 1u);
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_ts(tbase + kColDk, tbase + kColW + 16 + 8 * kk, adv(d_q_mn, 2048 * qt + 1024 * kk), id_mq,
-                   (qt > 0 || kk > 0) ? 1u : 0u);
-        });
       }
       if (!ok) break;
       if (threadIdx.x == 0 && i + 1 < nchunks) load_kv(i + 1);    // K, V no longer read

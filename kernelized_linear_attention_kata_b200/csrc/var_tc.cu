@@ -30,10 +30,20 @@
 //
 // Synchronous structure: 256 threads (two warps per TMEM lane quarter; half
 // h = warp / 4 splits the columns of each phase), thread 0 issues each round
-// of MMAs and commits it to one barrier every thread waits on.
+// of MMAs and commits it to one barrier every thread waits on. Independent
+// MMAs share rounds: per chunk
+//   1: U = Q Zd and the blocks of keys 0..63
+//   2: P V (keys 0..63, P in U's columns), the blocks of keys 64..127,
+//      readout groups 0, 1
+//   3: P V (keys 64..127), readout groups 2 (, 3), the update of state tiles
+//      0, 1 and Z
+//   4 (Mg2): readout group 4, the update of tile 2
+// (four rounds for Mg2, three for Sg2), the operands of the next round
+// written by the threads in between.
 //
 // Tensor memory (512 columns, fp32): S (NT tiles of 64 columns) | Z (32) |
-// U = Q Zd (32) | O (64) | work (the intra-chunk blocks, 64 keys at a time).
+// U = Q Zd, then P of keys 0..63 (32) | O (64) | work (the intra-chunk
+// blocks of 64 keys; Mg2 keeps P of keys 64..127 after them).
 #include "common.cuh"
 #include "launch.h"
 #include "profile.h"
@@ -74,11 +84,13 @@ struct VarSmem {
   static constexpr int V = 16384;              // [128][64] bf16, 128-byte swizzle
   static constexpr int Snap = 32768;           // S_c bf16 [384][64] (rows past D zero)
   static constexpr int ZSnap = Snap + 384 * 128;   // Zd bf16 [32][32]
-  static constexpr int Buf = ZSnap + 2048;     // 2 x 32 KB: key tiles, or 2 x 16 KB query slots
-  static constexpr int Lx = Buf + 65536;       // [128] fp32: half 1's partial l
+  static constexpr int Buf = ZSnap + 2048;     // 2 x 32 KB key-feature tiles (update A operand)
+  static constexpr int Slot = Buf + 65536;     // 2 x 16 KB query-feature slots (readout A operand)
+  static constexpr int Lx = Slot + 32768;      // [128] fp32: half 1's partial l
   static constexpr int Bars = Lx + 512;
   static constexpr int Bytes = Bars + 64 + 1024;
-  static_assert(Snap % 1024 == 0 && ZSnap % 1024 == 0 && Buf % 1024 == 0, "swizzle atoms");
+  static_assert(Snap % 1024 == 0 && ZSnap % 1024 == 0 && Buf % 1024 == 0 && Slot % 1024 == 0,
+                "swizzle atoms");
   static_assert(Bytes <= 232448, "shared memory budget");
 };
 enum { kVBarLoadQ = 0, kVBarLoadKV, kVBarMma, kVNumBars };
@@ -283,7 +295,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
   const uint64_t d_v_mn = smem_desc(smem_u32(smem + L::V), 16384, 1024, kSw128);  // MN-major
   const uint64_t d_snap = smem_desc(smem_u32(snap), 16384, 1024, kSw128);         // MN-major
   const uint64_t d_z = smem_desc(smem_u32(zsnap), 16, 512, kSw64);
-  const uint64_t d_slot = smem_desc(smem_u32(buf), 16, 1024, kSw128);             // K-major
+  const uint64_t d_slot = smem_desc(smem_u32(smem + L::Slot), 16, 1024, kSw128);   // K-major
   const uint64_t d_tile = smem_desc(smem_u32(buf), 16384, 1024, kSw128);          // MN-major
   constexpr uint32_t id_n64 = idesc_bf16(128, 64, false, false);
   constexpr uint32_t id_n32 = idesc_bf16(128, 32, false, false);
@@ -413,30 +425,99 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     const int c0 = t0 + i * kVC;
     const bool valid = c0 + r < T;
     if (!(ok = wait_all(&bars[kVBarLoadKV], i & 1))) break;
-    if (!AGG) {
+    // key tile M of the update (groups 2 M, 2 M + 1) into tile buffer tb
+    auto tile_groups = [&](auto mc, uint8_t *tb) {
+      constexpr int M = decltype(mc)::value;
+      uint32_t XK[16], Ka[16], Kb[16], w[32];
+      row_words(smem + L::K, r, XK);
+      half_pairs(XK, 0, Ka);
+      half_pairs(XK, 1, Kb);
+      if constexpr (2 * M < NG) {
+        group_words_c<V, true, 2 * M>(Ka, Kb, w);
+        store_words(tb, r, w);
+      }
+      if constexpr (2 * M + 1 < NG) {
+        group_words_c<V, true, 2 * M + 1>(Ka, Kb, w);
+        store_words(tb + 16384, r, w);
+      }
+    };
+    // S tile M += (tile buffer hb)^T V; Z += K^T K with the first tile
+    auto issue_update = [&](int M, int hb, bool with_z) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss(tbase + SH::ColS + 64 * M, adv(d_tile, 32768 * hb + 2048 * kk), adv(d_v_mn, 2048 * kk),
+               id_up, 1u);
+      if (with_z) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tbase + SH::ColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1u);
+      }
+    };
+
+    if constexpr (AGG) {
+      // ---- increment: the update only, two key tiles a round ----
+      auto update_round = [&](auto m0c) -> bool {
+        constexpr int M0 = decltype(m0c)::value;
+        if (half) {
+          if constexpr (M0 + 1 < NT) tile_groups(IC<M0 + 1>{}, buf + 32768);
+        } else {
+          tile_groups(IC<M0>{}, buf);
+        }
+        return round([&] {
+          issue_update(M0, 0, M0 == 0);
+          if constexpr (M0 + 1 < NT) issue_update(M0 + 1, 1, false);
+        });
+      };
+      ok = update_round(IC<0>{});
+      if constexpr (NT > 2) {
+        if (ok) ok = update_round(IC<2>{});
+      }
+      if (!ok) break;
+      if (threadIdx.x == 0 && i + 1 < nchunks) load_kv(i + 1);       // K, V no longer read
+      continue;
+    } else {
       if (!(ok = wait_all(&bars[kVBarLoadQ], i & 1))) break;
+      // the state after this chunk is needed by the next chunk, or returned
+      const bool upd = i < nchunks - 1 || state_out;
       uint32_t XQ[16], Pa[16], Pb[16];
       row_words(smem + L::Q, r, XQ);
       half_pairs(XQ, 0, Pa);
       half_pairs(XQ, 1, Pb);
-
-      // ---- intra-chunk: 64 keys at a time; P V into O ----
-      float l_part = 0.f, den_inter = 0.f;
-      for (int b = 0; ok && b < 2; ++b) {
-        ok = round([&] {
-          if (b == 0) {
+      // query-feature group G into this half's readout slot
+      auto slot_group = [&](auto gc) {
+        constexpr int G = decltype(gc)::value;
+        if constexpr (G < NG) {
+          uint32_t w[32];
+          group_words_c<V, false, G>(Pa, Pb, w);
+          store_words(smem + L::Slot + 16384 * (G & 1), r, w);
+        }
+      };
+      // O += slot (group G) x snapshot rows of group G
+      auto issue_readout = [&](int G) {
+        const int nk = G == NG - 1 ? 1 : 4;
+        for (int kk = 0; kk < nk; ++kk)
+          mma_ss(tbase + SH::ColO, adv(d_slot, 16384 * (G & 1) + 32 * kk),
+                 adv(d_snap, (64 * G + 16 * kk) * 128), id_ro, 1u);
+      };
+      // intra-chunk blocks Q_u K_w^T for keys 64 b .. 64 b + 63 into the work columns
+      auto issue_intra = [&](int b) {
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_ss(tbase + SH::ColU, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_n32, kk);
-          }
+        for (int j = 0; j < NA; ++j) {
+          // block (u, w): Mg2 (0,0), (1,1); Sg2 (0,0), (0,1), (1,0), (1,1)
+          const int u = V == kMg2 ? j : j >> 1, w = V == kMg2 ? j : j & 1;
+          mma_ss(tbase + SH::ColW + 64 * j, adv(d_q, 32 * u), adv(d_k, 4096 * b + 32 * w), id_n64, 0);
+        }
+      };
+      // P V for keys 64 b .. 64 b + 63, P (bf16) at column pc
+      auto issue_pv = [&](int b, uint32_t pc) {
 #pragma unroll
-          for (int j = 0; j < NA; ++j) {
-            // block (u, w): Mg2 (0,0), (1,1); Sg2 (0,0), (0,1), (1,0), (1,1)
-            const int u = V == kMg2 ? j : j >> 1, w = V == kMg2 ? j : j & 1;
-            mma_ss(tbase + SH::ColW + 64 * j, adv(d_q, 32 * u), adv(d_k, 4096 * b + 32 * w), id_n64, 0);
-          }
-        });
-        if (!ok) break;
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tbase + SH::ColO, tbase + pc + 8 * kk, adv(d_v_mn, 8192 * b + 2048 * kk), id_pv,
+                 (b > 0 || kk > 0) ? 1u : 0u);
+      };
+      // sum of squares of the blocks for this half's 32 keys, masked; P words
+      float l_part = 0.f;
+      auto weights = [&](int b, uint32_t (&p)[16]) {
         float wsum[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) wsum[c] = 0.f;
@@ -452,7 +533,6 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
           }
         }
         const int s0 = 64 * b + 32 * half;
-        uint32_t p[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const float w0 = s0 + 2 * c <= r ? wsum[2 * c] : 0.f;
@@ -460,11 +540,28 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
           l_part += w0 + w1;
           p[c] = pack_bf16x2(w0, w1);
         }
-        if (b == 0 && half == 0) {
+      };
+      // P of the second key half: Mg2 after its two blocks, Sg2 over its
+      // first block (read before the store)
+      constexpr uint32_t kColP1 = V == kMg2 ? SH::ColW + 128 : SH::ColW;
+      static_assert(V != kMg2 || SH::ColW + 160 <= kVTmemCols, "P of the second key half");
+
+      // round 1: U = Q Zd, the blocks of keys 0..63
+      ok = round([&] {
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+          mma_ss(tbase + SH::ColU, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_n32, kk);
+        issue_intra(0);
+      });
+      if (!ok) break;
+      float den_inter = 0.f;
+      {
+        uint32_t p[16];
+        weights(0, p);
+        if (half == 0) {
           uint32_t u[32];
           tmem_ld32(tbase + lane_off + SH::ColU, u);
           tmem_wait_ld();
-          // q . u over the row's 32 values
 #pragma unroll
           for (int w = 0; w < 16; ++w) {
             const float2 qq = bf2f(XQ[w]);
@@ -472,58 +569,56 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
             den_inter = fmaf(qq.y, __uint_as_float(u[2 * w + 1]), den_inter);
           }
         }
-        __syncthreads();           // every thread has read the blocks before P overwrites them
-        tmem_st16(tbase + lane_off + SH::ColW + 16 * half, p);
-        ok = round([&] {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tbase + SH::ColO, tbase + SH::ColW + 8 * kk, adv(d_v_mn, 8192 * b + 2048 * kk), id_pv,
-                   (b > 0 || kk > 0) ? 1u : 0u);
-        });
+        __syncthreads();       // U and the blocks are read: P of keys 0..63 goes to U's columns
+        tmem_st16(tbase + lane_off + SH::ColU + 16 * half, p);
       }
+      if (half) slot_group(IC<1>{}); else slot_group(IC<0>{});
+      // round 2: P V (keys 0..63), the blocks of keys 64..127, readout groups 0, 1
+      ok = round([&] {
+        issue_pv(0, SH::ColU);
+        issue_intra(1);
+        issue_readout(0);
+        issue_readout(1);
+      });
       if (!ok) break;
-
-      // ---- readout: O += phi_q(Q) S_c, two 64-feature groups a round (half
-      //      0 writes group G0 into slot 0, half 1 group G0 + 1 into slot 1;
-      //      the last group is one K-step of 16 rows) ----
-      auto readout_round = [&](auto g0c) -> bool {
-        constexpr int G0 = decltype(g0c)::value;
-        uint32_t w[32];
-        if (half) {
-          if constexpr (G0 + 1 < NG) {
-            group_words_c<V, false, G0 + 1>(Pa, Pb, w);
-            store_words(buf + 16384, r, w);
-          }
-        } else {
-          group_words_c<V, false, G0>(Pa, Pb, w);
-          store_words(buf, r, w);
+      {
+        uint32_t p[16];
+        weights(1, p);
+        __syncthreads();       // every thread has read the blocks
+        tmem_st16(tbase + lane_off + kColP1 + 16 * half, p);
+      }
+      if (half) lx[r] = l_part;
+      if (half) slot_group(IC<3>{}); else slot_group(IC<2>{});
+      if (upd) {
+        if (half) tile_groups(IC<1>{}, buf + 32768); else tile_groups(IC<0>{}, buf);
+      }
+      // round 3: P V (keys 64..127), readout groups 2, 3, update of tiles 0, 1 and Z
+      ok = round([&] {
+        issue_pv(1, kColP1);
+        issue_readout(2);
+        if (NG > 4) issue_readout(3);
+        if (upd) {
+          issue_update(0, 0, true);
+          issue_update(1, 1, false);
         }
-        return round([&] {
-          constexpr int nk0 = G0 == NG - 1 ? 1 : 4;
-#pragma unroll
-          for (int kk = 0; kk < nk0; ++kk)
-            mma_ss(tbase + SH::ColO, adv(d_slot, 32 * kk), adv(d_snap, (64 * G0 + 16 * kk) * 128),
-                   id_ro, 1u);
-          if constexpr (G0 + 1 < NG) {
-            constexpr int nk1 = G0 + 1 == NG - 1 ? 1 : 4;
-#pragma unroll
-            for (int kk = 0; kk < nk1; ++kk)
-              mma_ss(tbase + SH::ColO, adv(d_slot, 16384 + 32 * kk),
-                     adv(d_snap, (64 * (G0 + 1) + 16 * kk) * 128), id_ro, 1u);
-          }
-        });
-      };
-      ok = readout_round(IC<0>{});
-      if (ok) ok = readout_round(IC<2>{});
-      if constexpr (NG > 4) {
-        if (ok) ok = readout_round(IC<4>{});
-      }
+      });
       if (!ok) break;
-      if (threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);        // Q no longer read
+      if constexpr (NG > 4) {
+        // round 4 (Mg2): readout group 4, update of tile 2
+        if (!half) slot_group(IC<4>{});
+        if (upd && !half) tile_groups(IC<2>{}, buf);
+        ok = round([&] {
+          issue_readout(4);
+          if (upd) issue_update(2, 0, false);
+        });
+        if (!ok) break;
+      }
+      if (threadIdx.x == 0 && i + 1 < nchunks) {
+        load_q(i + 1);                                           // Q, K, V no longer read
+        load_kv(i + 1);
+      }
 
       // ---- y = O / (l + q^T Zd q) ----
-      if (half) lx[r] = l_part;
-      __syncthreads();
       if (!half) {
         const float den = l_part + lx[r] + den_inter;
         if (valid && !(den > 0.f)) flag_status(status, kStatusNonPositiveNormaliser);
@@ -541,61 +636,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
           }
         }
       }
-    }
-    if (!AGG && i == nchunks - 1 && !state_out) break;
-
-    // ---- update: S += phi(K)^T V (two tiles a round), Z += K^T K ----
-    {
-      uint32_t XK[16], Pa[16], Pb[16];
-      row_words(smem + L::K, r, XK);
-      half_pairs(XK, 0, Pa);
-      half_pairs(XK, 1, Pb);
-      // half 0 writes tile M0 (groups 2 M0, 2 M0 + 1), half 1 tile M0 + 1
-      auto tile_groups = [&](auto mc, uint8_t *tb) {
-        constexpr int M = decltype(mc)::value;
-        uint32_t w[32];
-        if constexpr (2 * M < NG) {
-          group_words_c<V, true, 2 * M>(Pa, Pb, w);
-          store_words(tb, r, w);
-        }
-        if constexpr (2 * M + 1 < NG) {
-          group_words_c<V, true, 2 * M + 1>(Pa, Pb, w);
-          store_words(tb + 16384, r, w);
-        }
-      };
-      auto update_round = [&](auto m0c) -> bool {
-        constexpr int M0 = decltype(m0c)::value;
-        if (half) {
-          if constexpr (M0 + 1 < NT) tile_groups(IC<M0 + 1>{}, buf + 32768);
-        } else {
-          tile_groups(IC<M0>{}, buf);
-        }
-        return round([&] {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + SH::ColS + 64 * M0, adv(d_tile, 2048 * kk), adv(d_v_mn, 2048 * kk), id_up, 1u);
-          if constexpr (M0 + 1 < NT) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tbase + SH::ColS + 64 * (M0 + 1), adv(d_tile, 32768 + 2048 * kk),
-                     adv(d_v_mn, 2048 * kk), id_up, 1u);
-          }
-          if constexpr (M0 == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tbase + SH::ColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1u);
-          }
-        });
-      };
-      ok = update_round(IC<0>{});
-      if constexpr (NT > 2) {
-        if (ok) ok = update_round(IC<2>{});
-      }
-      if (!ok) break;
-      if (threadIdx.x == 0 && i + 1 < nchunks) load_kv(i + 1);       // K, V no longer read
-    }
-    // ---- snapshot S_c+1 and Zd_c+1 (not after the last chunk) ----
-    if constexpr (!AGG) {
+      // ---- snapshot S_c+1 and Zd_c+1 (not after the last chunk) ----
       if (i < nchunks - 1) {
         for (int mt = half; mt < NT; mt += 2) {
           const int f = 128 * mt + r;
