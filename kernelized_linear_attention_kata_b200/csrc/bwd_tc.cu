@@ -190,7 +190,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
   // MMAs and commits them, every thread waits. The result is uniform over
   // the CTA, so a timeout ends every thread's loop at the same point.
   uint32_t mph = 0;
-  auto round = [&](auto issue) -> bool {
+  // round_with also runs CUDA-core work while the MMAs are in flight: work
+  // that neither reads nor writes what they touch.
+  auto round_with = [&](auto issue, auto work) -> bool {
     tmem_wait_ld();
     tmem_wait_st();
     fence_async_smem();
@@ -201,11 +203,13 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
       issue();
       mma_commit(&bars[kBarMma]);
     }
+    work();
     const bool ok = mbar_wait(&bars[kBarMma], mph, abort_flag);
     mph ^= 1;
     tc_fence_after();
     return __syncthreads_and(ok);
   };
+  auto round = [&](auto issue) -> bool { return round_with(issue, [] {}); };
   auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
     return __syncthreads_and(mbar_wait(bar, parity, abort_flag));
   };
@@ -405,7 +409,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
 #pragma unroll
     for (int l = 0; l < 32; ++l) h[l] += g2R[l];
 
-    // ---- combine the halves: d_t, c_t, the carried dq ----
+    // ---- combine the halves (d_t, c_t, the carried dq) while the intra
+    //      blocks of keys 0..63 are recomputed; then M = 2 A (D' / d_t + c_t)
+    //      masked, dq += M K_b ----
     if (half) {
       float *row = xch + r * 36;
       row[32] = l_part;
@@ -414,34 +420,36 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
       for (int l = 0; l < 32; l += 4)
         *reinterpret_cast<float4 *>(row + l) = make_float4(h[l], h[l + 1], h[l + 2], h[l + 3]);
     }
-    __syncthreads();
     float dqc[32];
-    if (!half) {
-      const float *row = xch + r * 36;
-      const float l_all = l_part + row[32];
-      const float dn_all = dn_part + dn_car + row[33];
-      const float d = l_all + den_inter;
-      if (valid && !(d > 0.f)) flag_status(status, kStatusNonPositiveNormaliser);
-      const float inv = valid ? 1.f / d : 0.f;
-      const float ct = valid ? -dn_all * inv * inv : 0.f;
-      invd_s[r] = inv;
-      c_s[r] = ct;
-      if (valid) {
-        den_out[(size_t)bh * T + c0 + r] = d;
-        c_out[(size_t)bh * T + c0 + r] = ct;
-      }
-      const float *u = ubuf + r * 32;
+    auto combine = [&] {        // half 1's partial sums are in xch (the round's barrier)
+      if (!half) {
+        const float *row = xch + r * 36;
+        const float l_all = l_part + row[32];
+        const float dn_all = dn_part + dn_car + row[33];
+        const float d = l_all + den_inter;
+        if (valid && !(d > 0.f)) flag_status(status, kStatusNonPositiveNormaliser);
+        const float inv = valid ? 1.f / d : 0.f;
+        const float ct = valid ? -dn_all * inv * inv : 0.f;
+        invd_s[r] = inv;
+        c_s[r] = ct;
+        if (valid) {
+          den_out[(size_t)bh * T + c0 + r] = d;
+          c_out[(size_t)bh * T + c0 + r] = ct;
+        }
+        const float *u = ubuf + r * 32;
 #pragma unroll
-      for (int l = 0; l < 32; ++l) dqc[l] = inv * (h[l] + row[l]) + 2.f * ct * u[l];
-    }
-    __syncthreads();
-
-    // ---- intra-chunk dq: M = 2 A (D' / d_t + c_t) masked, dq += M K_b ----
-    const float inv_r = invd_s[r], c_r = c_s[r];
+        for (int l = 0; l < 32; ++l) dqc[l] = inv * (h[l] + row[l]) + 2.f * ct * u[l];
+      }
+    };
     for (int b = 0; ok && b < 2; ++b) {
-      ok = round([&] { issue_intra(b); });
+      if (b == 0) {
+        ok = round_with([&] { issue_intra(0); }, combine);
+      } else {
+        ok = round([&] { issue_intra(1); });
+      }
       if (!ok) break;
       if (b == 1 && threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);   // Q, dout read
+      const float inv_r = invd_s[r], c_r = c_s[r];
       uint32_t a[32], dp[32], m[16];
       tmem_ld32(tbase + lane_off + kColA + 32 * half, a);
       tmem_ld32(tbase + lane_off + kColB + 32 * half, dp);
@@ -466,23 +474,27 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
       });
     }
     if (!ok) break;
-    if (!half) {
-      uint32_t acc[32];
-      tmem_ld32(tbase + lane_off + kColDq, acc);
-      tmem_wait_ld();
-      if (valid) {
-        uint4 *dst = reinterpret_cast<uint4 *>(dq + ((size_t)bh * T + c0 + r) * kDK);
+    // dq = the intra part (tensor memory) + the carried part (half 0)
+    auto write_dq = [&] {
+      if (!half) {
+        uint32_t acc[32];
+        tmem_ld32(tbase + lane_off + kColDq, acc);
+        tmem_wait_ld();
+        if (valid) {
+          uint4 *dst = reinterpret_cast<uint4 *>(dq + ((size_t)bh * T + c0 + r) * kDK);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t w[4];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            w[j] = pack_bf16x2(__uint_as_float(acc[8 * c + 2 * j]) + dqc[8 * c + 2 * j],
-                               __uint_as_float(acc[8 * c + 2 * j + 1]) + dqc[8 * c + 2 * j + 1]);
-          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int j = 0; j < 4; ++j)
+              w[j] = pack_bf16x2(__uint_as_float(acc[8 * c + 2 * j]) + dqc[8 * c + 2 * j],
+                                 __uint_as_float(acc[8 * c + 2 * j + 1]) + dqc[8 * c + 2 * j + 1]);
+            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
-    }
+    };
+    write_dq();
     if (i == nchunks - 1) break;            // the state after the segment is not needed
 
     // ---- update: S += phi(K)^T V, Z += K^T K; three rounds of two key tiles ----
@@ -503,7 +515,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
         } else {
           rotate_left(R2, 4);
         }
-        ok = round([&] {
+        auto issue_upd = [&] {
           const int ma = u < 2 ? u : 4, mb = 2 + u;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -519,7 +531,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tbase + kColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1);
           }
-        });
+        };
+        ok = round(issue_upd);
       }
       if (!ok) break;
       if (threadIdx.x == 0) load_kv(i + 1);           // K, V of this chunk no longer read
@@ -681,7 +694,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
   }
 
   uint32_t mph = 0;
-  auto round = [&](auto issue) -> bool {
+  // round_with also runs CUDA-core work while the MMAs are in flight: work
+  // that neither reads nor writes what they touch.
+  auto round_with = [&](auto issue, auto work) -> bool {
     tmem_wait_ld();
     tmem_wait_st();
     fence_async_smem();
@@ -692,11 +707,13 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
       issue();
       mma_commit(&bars[kBarMma]);
     }
+    work();
     const bool ok = mbar_wait(&bars[kBarMma], mph, abort_flag);
     mph ^= 1;
     tc_fence_after();
     return __syncthreads_and(ok);
   };
+  auto round = [&](auto issue) -> bool { return round_with(issue, [] {}); };
   auto wait_all = [&](uint64_t *bar, uint32_t parity) -> bool {
     return __syncthreads_and(mbar_wait(bar, parity, abort_flag));
   };
@@ -788,17 +805,68 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     }
   }
 
+  // d_t and c_t of a chunk (threads 0..127, one token each), loaded a chunk
+  // ahead so that the load's latency hides behind the chunk's work
+  float pf_den = 1.f, pf_c = 0.f;
+  auto fetch_dc = [&](int i) {
+    const int t = t0 + chunk_of(i) * kC + (int)threadIdx.x;
+    if (threadIdx.x < kC && t < T) {
+      pf_den = den[(size_t)bh * T + t];
+      pf_c = cvec[(size_t)bh * T + t];
+    } else {
+      pf_den = 0.f;
+      pf_c = 0.f;
+    }
+  };
+  if (nchunks > 0) fetch_dc(0);
+
   bool ok = true;
   for (int i = 0; ok && i < nchunks; ++i) {
     const int c0 = t0 + chunk_of(i) * kC;
     const bool valid = c0 + r < T;
+    // dk = the intra part + the carried part from ubuf (half 0); dv (half 1)
+    auto write_outputs = [&] {
+      if constexpr (!AGG) {
+        if (!half) {
+          uint32_t acc[32];
+          tmem_ld32(tbase + lane_off + kColDk, acc);
+          tmem_wait_ld();
+          const float *u = ubuf + r * 32;
+          if (valid) {
+            uint4 *dst = reinterpret_cast<uint4 *>(dk + ((size_t)bh * T + c0 + r) * kDK);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t w[4];
+#pragma unroll
+              for (int j2 = 0; j2 < 4; ++j2) {
+                const int l0 = 8 * c + 2 * j2;
+                w[j2] = pack_bf16x2(__uint_as_float(acc[l0]) + u[l0],
+                                    __uint_as_float(acc[l0 + 1]) + u[l0 + 1]);
+              }
+              dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        } else {
+          uint32_t acc[32];
+#pragma unroll 1
+          for (int hv = 0; hv < 2; ++hv) {
+            tmem_ld32(tbase + lane_off + kColDv + 32 * hv, acc);
+            tmem_wait_ld();
+            if (valid) {
+              uint4 *dst = reinterpret_cast<uint4 *>(dv + ((size_t)bh * T + c0 + r) * kDV + 32 * hv);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) dst[c] = pack8(acc + 8 * c);
+            }
+          }
+        }
+      }
+    };
     if (!(ok = wait_all(&bars[kBarLoadQ], i & 1))) break;
     if (threadIdx.x < kC) {
-      const int t = c0 + threadIdx.x;
-      const bool vt = t < T;
-      invd_s[threadIdx.x] = vt ? 1.f / den[(size_t)bh * T + t] : 0.f;
-      c_s[threadIdx.x] = vt ? cvec[(size_t)bh * T + t] : 0.f;
+      invd_s[threadIdx.x] = pf_den != 0.f ? 1.f / pf_den : 0.f;
+      c_s[threadIdx.x] = pf_c;
     }
+    if (i + 1 < nchunks) fetch_dc(i + 1);
     __syncthreads();
     if (!AGG) {
       if (!(ok = wait_all(&bars[kBarLoadKV], i & 1))) break;
@@ -919,7 +987,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         const uint32_t ws_col = kColW + 8 * half;           // this half's W~ words
         const uint32_t ms_col = kColW + 16 + 8 * half;      // this half's M words
         for (int qt = 0; ok && qt < 4; ++qt) {
-          ok = round([&] {
+          // the first round also folds the carried dk into ubuf: J(k)^T Y of
+          // both halves (half 1's from xch) plus 2 Rq k
+          ok = round_with([&] {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk)
               mma_ss(tbase + kColW, adv(d_k, 32 * kk), adv(d_q, 2048 * qt + 32 * kk), id_n32, kk);
@@ -927,6 +997,13 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
             for (int kk = 0; kk < 4; ++kk)
               mma_ss(tbase + kColW + 32, adv(d_v, 32 * kk), adv(d_o, 4096 * qt + 32 * kk), id_n32, kk);
             issue_slots(qt);
+          }, [&] {
+            if (qt == 0 && !half) {
+              const float *row = xch + r * 36;
+              float *u = ubuf + r * 32;
+#pragma unroll
+              for (int l = 0; l < 32; ++l) u[l] = h[l] + row[l] + 2.f * u[l];
+            }
           });
           if (!ok) break;
           uint32_t a[16], dp[16], wv[8], mv[8];
@@ -952,8 +1029,11 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
           __syncthreads();        // every thread has read its columns before W~, M overwrite them
           tmem_st8(tbase + lane_off + ws_col, wv);
           tmem_st8(tbase + lane_off + ms_col, mv);
-          write_slot(qt + 1);     // the previous pair's slots were read by the last round
-          ok = round([&] {
+          // the next slot pair is written while this round runs (the last
+          // round read the previous pair); the last pair, read by the last
+          // round, before it
+          if (qt == 3) write_slot(4);
+          ok = round_with([&] {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk)
               mma_ts(tbase + kColDv, tbase + kColW + 8 * kk, adv(d_o_mn, 4096 * qt + 2048 * kk), id_wo,
@@ -963,46 +1043,18 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
               mma_ts(tbase + kColDk, tbase + kColW + 16 + 8 * kk, adv(d_q_mn, 2048 * qt + 1024 * kk),
                      id_mq, (qt > 0 || kk > 0) ? 1u : 0u);
             if (qt == 3) issue_slots(4);
+          }, [&] {
+            if (qt < 3) write_slot(qt + 1);
           });
         }
       }
       if (!ok) break;
       if (threadIdx.x == 0 && i + 1 < nchunks) load_kv(i + 1);    // K, V no longer read
-      // ---- outputs: dk = intra + J(k)^T Y + 2 Rq k (half 0), dv (half 1) ----
-      if (!half) {
-        uint32_t acc[32];
-        tmem_ld32(tbase + lane_off + kColDk, acc);
-        tmem_wait_ld();
-        const float *row = xch + r * 36, *u = ubuf + r * 32;
-        if (valid) {
-          uint4 *dst = reinterpret_cast<uint4 *>(dk + ((size_t)bh * T + c0 + r) * kDK);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j2 = 0; j2 < 4; ++j2) {
-              const int l0 = 8 * c + 2 * j2;
-              w[j2] = pack_bf16x2(__uint_as_float(acc[l0]) + h[l0] + row[l0] + 2.f * u[l0],
-                                  __uint_as_float(acc[l0 + 1]) + h[l0 + 1] + row[l0 + 1] + 2.f * u[l0 + 1]);
-            }
-            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      } else {
-        uint32_t acc[32];
-#pragma unroll 1
-        for (int hv = 0; hv < 2; ++hv) {
-          tmem_ld32(tbase + lane_off + kColDv + 32 * hv, acc);
-          tmem_wait_ld();
-          if (valid) {
-            uint4 *dst = reinterpret_cast<uint4 *>(dv + ((size_t)bh * T + c0 + r) * kDV + 32 * hv);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) dst[c] = pack8(acc + 8 * c);
-          }
-        }
-      }
     }
-    if (!AGG && i == nchunks - 1) break;       // the state before the segment is not needed
+    if (!AGG && i == nchunks - 1) {            // the state before the segment is not needed
+      write_outputs();
+      break;
+    }
 
     // ---- update: R' += (m p(q) / d)^T dout (tiles (0, 2), (1, 3), (4)), Rq += Q^T diag(c) Q ----
     {
@@ -1034,7 +1086,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         } else {
           rotate_left(R2, 4);
         }
-        ok = round([&] {
+        auto issue_upd = [&] {
           const int ma = u < 2 ? u : 4, mb = 2 + u;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -1050,7 +1102,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tbase + kColRq, adv(d_cq, 1024 * kk), adv(d_q_mn, 1024 * kk), id_rq, 1);
           }
-        });
+        };
+        // dk and dv leave while the first update round runs (it touches neither)
+        ok = u == 0 ? round_with(issue_upd, write_outputs) : round(issue_upd);
       }
       if (!ok) break;
       if (threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);     // Q, dout no longer read
