@@ -67,6 +67,8 @@ CASES = [
     # with a ragged last chunk, and segments of several chunks
     ("psd", "bf16", 1, 3, 1000, 32, 64, 128),
     ("psd", "bf16", 2, 20, 2000, 32, 64, 128),
+    ("psd", "bf16", 1, 1, 1, 32, 64, 128),
+    ("psd", "bf16", 1, 2, 129, 32, 64, 64),
     ("first_order", "f32", 1, 1, 1, 64, 64, 64),
     ("first_order", "f32", 1, 2, 191, 64, 64, 64),
     ("first_order", "f32", 2, 2, 100, 16, 32, 32),
