@@ -140,6 +140,8 @@ KERNEL_SOURCES = {
     "tc_bwd_dq": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
     "tc_bwd_dkdv": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
     "tc_bwd_suffix_increment": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
+    "tc_variant_pass": ["var_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
+    "tc_variant_increment": ["var_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
 }
 
 
