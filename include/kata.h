@@ -147,7 +147,9 @@ KATA_API int kata_version(void);
 KATA_API const char *kata_status_string(kata_status_t status);
 
 /* D, the number of state rows: d_k (d_k + 1) / 2 for PSD, d_k + 1 for
- * FIRST_ORDER; 0 for an unknown feature or d_k <= 0. */
+ * FIRST_ORDER, h (h + 1) for MULTI_PSD2 and h (h + 1) / 2 for SUMMED_PSD2
+ * (h = d_k / 2); 0 for an unknown feature, d_k <= 0, or an odd d_k with a
+ * two-factor feature. */
 KATA_API size_t kata_state_dim(int d_k, kata_feature_t feature);
 
 /*
