@@ -362,7 +362,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": base.cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -391,10 +391,10 @@ def aggregate_throughput(ms_per_step, tokens_per_step, world, device):
     return world * tokens_per_step / (ms / 1e3), ms
 
 
-def workload_config(w):
+def workload_config(w, world=1):
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d_k": w.d_k, "d_v": w.d_v,
             "C": w.C, "feature": w.feature, "form": "chunked (segmented scan carry)",
-            "l2": "inputs larger than L2 (no flush needed)", "parallelism": "replicas"}
+            "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{world}"}
 
 
 # ---------------------------------------------------------------------------
