@@ -36,6 +36,10 @@
 // written out. Math thread r owns TMEM lane r (quarter = warp mod 4):
 // token r of the chunk for the token-major tiles, feature row r of each
 // 128-feature state tile.
+// The increment kernel (AGG) has no query side: warps 2-5 write the key
+// features of tiles 1 and 3 and warps 6-9 those of tiles 0, 2 and 4, and
+// the two update issuers (warp 1: Z and tiles 1, 3; warp 10: tiles 0, 2, 4)
+// each consume one set, so that both sets and both issuers work at once.
 //
 // Tensor memory (512 columns, fp32):
 //   [  0, 320)  S, five 128-feature tiles of 64 columns (tile 4: 16 rows used)
@@ -150,7 +154,8 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     mbar_init(&bars[kBarQEmpty], 1 + A);            // Q K^T commit + query side
     for (int st = 0; st < 2; ++st) {
       mbar_init(&bars[kBarKvFull + st], 1);
-      mbar_init(&bars[kBarKvEmpty + st], 2 + A);      // two MMA warps + key side
+      // two MMA warps + key side (+ the second feature set of the increment kernel)
+      mbar_init(&bars[kBarKvEmpty + st], AGG ? 2 + 2 * A : 2 + A);
     }
     mbar_init(&bars[kBarSFull], 1);
     mbar_init(&bars[kBarPFull], A);
@@ -348,7 +353,8 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       } else if (warp == 10 || (AGG && warp == 1)) {
         // ---------------- state-side MMAs ----------------
         // In the increment kernel (no readout) warps 10 and 1 split the
-        // tiles (warp 10: Z and tiles 0, 2, 4; warp 1: tiles 1, 3).
+        // tiles (warp 10: tiles 0, 2, 4; warp 1: Z and tiles 1, 3), as the
+        // two feature sets split their production.
         // The key side writes the key features of chunk i after its snapshots
         // of S_i and Z_i (and after K_i, V_i arrived), so a full key-ring slot
         // also says that the state it updates has been read.
@@ -359,7 +365,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const int u = i * kTiles + m, b = u % NK;
             if (!(ok = mbar_wait(&bars[kBarKRingFull + b], (u / NK) & 1, abort_flag))) break;
             tc_fence_after();
-            if (m == 0) {
+            if (m == (AGG ? 1 : 0)) {
               // Z += K^T K (A rows 32..127 alias other shared memory; unused lanes)
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
@@ -544,6 +550,29 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         fence_async_smem();
         warp_arrive(&bars[kBarStageFull]);          // warp 11 stores the tile
       }
+    } else {
+      // ---- increment kernel: the key features of tiles 1 and 3, so that
+      //      two feature sets (and both issuing warps) work at once ----
+      const int r = (warp & 3) * 32 + lane;               // token of the chunk
+      // the key side zeroes the accumulators first (its Z-snapshot arrival)
+      bool ok = warp_wait(&bars[kBarZSnap], 0, abort_flag);
+      for (int i = 0; ok && i < nchunks; ++i) {
+        const int st = i & 1;
+        if (!(ok = warp_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
+        uint32_t XK[16], P[32], R2[32];
+        load_pairs(smem + L::kOffK + 8192 * st, r, XK, P);
+        warp_arrive(&bars[kBarKvEmpty + st]);           // K rows read
+#pragma unroll
+        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[(l + 4) & 31], 0x40004000u);   // x 2, rotated by 4
+#pragma unroll 1
+        for (int m = 1; m < kTiles; m += 2) {
+          const int u = i * kTiles + m;
+          if (!(ok = ring_acquire(&bars[kBarKRingEmpty], NK, u))) break;
+          write_tile(kring + (u % NK) * kKSlotBytes, r, false, 0x3f803f80u, P, R2);
+          ring_publish(&bars[kBarKRingFull], NK, u);
+          rotate_left(R2, 8);
+        }
+      }
     }
   } else if (warp < 10) {
     // -------------------------------------------------- key side (warps 6..9)
@@ -654,8 +683,9 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll 1
         for (int m = 0; m < kTiles; ++m) {
           const int u = i * kTiles + m;
-          if (ok) ok = ring_acquire(&bars[kBarKRingEmpty], NK, u);
-          if (ok) {
+          const bool mine = !AGG || (m & 1) == 0;        // increments: tiles 1, 3 go to warps 2..5
+          if (ok && mine) ok = ring_acquire(&bars[kBarKRingEmpty], NK, u);
+          if (ok && mine) {
             write_tile(kring + (u % NK) * kKSlotBytes, r, m == kTiles - 1,
                        m == 0 ? 0x3f003f00u : 0x3f803f80u, P, R2);     // x 1/2 on the diagonal
             ring_publish(&bars[kBarKRingFull], NK, u);
