@@ -30,8 +30,10 @@
 // 0 .. g-1 as its carry-in; each CTA then walks its segment's chunks.
 //
 // The kernel is synchronous: 256 threads (8 warps, two per TMEM lane
-// quarter; "half" h = warp / 4 splits each phase's columns), thread 0 issues
-// a round of MMAs and commits them to one barrier that every thread waits
+// quarter; "half" h = warp / 4 splits each phase's columns). Threads 0 and
+// 32 issue a round of MMAs, each accumulator's chain from one of them (one
+// thread issues an N <= 64 MMA only every 75-100 cycles, so two issue about
+// twice as fast), and commit them to one barrier that every thread waits
 // on. The state, the feature order and its doubled off-diagonal rows are
 // the forward's (psd_tc_common.cuh).
 //
@@ -153,7 +155,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarLoadQ], 1);
     mbar_init(&bars[kBarLoadKV], 1);
-    mbar_init(&bars[kBarMma], 1);
+    mbar_init(&bars[kBarMma], 2);                 // one commit per issuing thread
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -186,8 +188,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
   }
 
   // One synchronous round: every thread's operand writes (shared memory,
-  // tensor memory) and tensor-memory reads are complete, thread 0 issues the
-  // MMAs and commits them, every thread waits. The result is uniform over
+  // tensor memory) and tensor-memory reads are complete, threads 0 and 32
+  // issue the MMAs (issue(0), issue(1): every accumulator's MMAs from one of
+  // them) and commit them, every thread waits. The result is uniform over
   // the CTA, so a timeout ends every thread's loop at the same point.
   uint32_t mph = 0;
   // round_with also runs CUDA-core work while the MMAs are in flight: work
@@ -198,9 +201,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 || threadIdx.x == 32) {
       tc_fence_after();
-      issue();
+      issue(threadIdx.x >> 5);
       mma_commit(&bars[kBarMma]);
     }
     work();
@@ -233,13 +236,16 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
   constexpr uint32_t id_z = idesc_bf16(128, 32, true, true);
 
   // A = Q K_b^T and D' = dout V_b^T for keys 64 b .. 64 b + 63
-  auto issue_intra = [&](int b) {
+  auto issue_intra = [&](int b, int who) {
+    if (who == 0) {
 #pragma unroll
-    for (int kk = 0; kk < 2; ++kk)
-      mma_ss(tbase + kColA, adv(d_q, 32 * kk), adv(d_k, 4096 * b + 32 * kk), id_n64, kk);
+      for (int kk = 0; kk < 2; ++kk)
+        mma_ss(tbase + kColA, adv(d_q, 32 * kk), adv(d_k, 4096 * b + 32 * kk), id_n64, kk);
+    } else {
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_v, 8192 * b + 32 * kk), id_n64, kk);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_v, 8192 * b + 32 * kk), id_n64, kk);
+    }
   };
 
   // ---- carry-in: S, Z = the increments of segments 0 .. g-1 ----
@@ -318,13 +324,13 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
     // ---- intra-chunk row sums: l = sum_s w_ts, dn = sum_s w_ts (dout_t . v_s) ----
     float l_part = 0.f, dn_part = 0.f, den_inter = 0.f;
     for (int b = 0; ok && b < 2; ++b) {
-      ok = round([&] {
-        if (b == 0) {
+      ok = round([&](int who) {
+        if (b == 0 && who == 0) {
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
             mma_ss(tbase + kColDq, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_n32, kk);
         }
-        issue_intra(b);
+        issue_intra(b, who);
       });
       if (!ok) break;
       uint32_t a[32], dp[32];
@@ -368,16 +374,17 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
     if (half) rot<8>(qR);
     float dn_car = 0.f;
     for (int j = 0; ok && j < 5; ++j) {
-      ok = round([&] {
-        if (j < 4) {
+      ok = round([&](int who) {
+        if (j < 4 && who == 0) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tbase + kColA, adv(d_o, 32 * kk), adv(d_snap, 64 * j * 128 + 32 * kk), id_n64, kk);
+        } else if (j < 4) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_snap, (256 + 64 * j) * 128 + 32 * kk),
                    id_n64, kk);
-        } else {
+        } else if (who == 1) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
@@ -443,9 +450,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
     };
     for (int b = 0; ok && b < 2; ++b) {
       if (b == 0) {
-        ok = round_with([&] { issue_intra(0); }, combine);
+        ok = round_with([&](int who) { issue_intra(0, who); }, combine);
       } else {
-        ok = round([&] { issue_intra(1); });
+        ok = round([&](int who) { issue_intra(1, who); });
       }
       if (!ok) break;
       if (b == 1 && threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);   // Q, dout read
@@ -466,7 +473,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
       }
       __syncthreads();          // every thread has read A and D' before M overwrites A
       tmem_st16(tbase + lane_off + kColA + 16 * half, m);
-      ok = round([&] {
+      ok = round([&](int who) {
+        if (who != 0) return;                    // one accumulator: one issuing thread
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_ts(tbase + kColDq, tbase + kColA + 8 * kk, adv(d_k_mn, 4096 * b + 1024 * kk), id_mk,
@@ -515,18 +523,20 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
         } else {
           rotate_left(R2, 4);
         }
-        auto issue_upd = [&] {
+        auto issue_upd = [&](int who) {
           const int ma = u < 2 ? u : 4, mb = 2 + u;
+          if (who == 0) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + kColS + 64 * ma, adv(d_key, 2048 * kk), adv(d_v_mn, 2048 * kk), id_up, 1);
-          if (u < 2) {
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + kColS + 64 * ma, adv(d_key, 2048 * kk), adv(d_v_mn, 2048 * kk), id_up, 1);
+          }
+          if (u < 2 && who == 1) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tbase + kColS + 64 * mb, adv(d_key, 32768 + 2048 * kk), adv(d_v_mn, 2048 * kk),
                      id_up, 1);
           }
-          if (u == 0) {
+          if (u == 0 && who == 0) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tbase + kColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1);
@@ -657,7 +667,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarLoadQ], 1);
     mbar_init(&bars[kBarLoadKV], 1);
-    mbar_init(&bars[kBarMma], 1);
+    mbar_init(&bars[kBarMma], 2);                 // one commit per issuing thread
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -702,9 +712,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 || threadIdx.x == 32) {
       tc_fence_after();
-      issue();
+      issue(threadIdx.x >> 5);
       mma_commit(&bars[kBarMma]);
     }
     work();
@@ -884,22 +894,23 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
       if (half) rot<8>(kR);
       float unused = 0.f;
       for (int j = 0; ok && j < 5; ++j) {
-        ok = round([&] {
-          if (j == 0) {
+        ok = round([&](int who) {
+          if (j == 0 && who == 0) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk)
               mma_ss(tbase + kColDk, adv(d_k, 32 * kk), adv(d_rq, 32 * kk), id_n32, kk);
           }
-          if (j < 4) {
+          if (j < 4 && who == 0) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_ss(tbase + kColDv, adv(d_v, 32 * kk), adv(d_snap, 64 * j * 128 + 32 * kk), id_n64,
                      kk);
+          } else if (j < 4) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_ss(tbase + kColW, adv(d_v, 32 * kk), adv(d_snap, (256 + 64 * j) * 128 + 32 * kk),
                      id_n64, kk);
-          } else {
+          } else if (who == 1) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_ss(tbase + kColW, adv(d_v, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
@@ -989,14 +1000,17 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         for (int qt = 0; ok && qt < 4; ++qt) {
           // the first round also folds the carried dk into ubuf: J(k)^T Y of
           // both halves (half 1's from xch) plus 2 Rq k
-          ok = round_with([&] {
+          ok = round_with([&](int who) {
+            if (who == 0) {
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_ss(tbase + kColW, adv(d_k, 32 * kk), adv(d_q, 2048 * qt + 32 * kk), id_n32, kk);
+              for (int kk = 0; kk < 2; ++kk)
+                mma_ss(tbase + kColW, adv(d_k, 32 * kk), adv(d_q, 2048 * qt + 32 * kk), id_n32, kk);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ss(tbase + kColW + 32, adv(d_v, 32 * kk), adv(d_o, 4096 * qt + 32 * kk), id_n32, kk);
-            issue_slots(qt);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tbase + kColW + 32, adv(d_v, 32 * kk), adv(d_o, 4096 * qt + 32 * kk), id_n32, kk);
+            } else {
+              issue_slots(qt);                     // the dv accumulator
+            }
           }, [&] {
             if (qt == 0 && !half) {
               const float *row = xch + r * 36;
@@ -1033,16 +1047,19 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
           // round read the previous pair); the last pair, read by the last
           // round, before it
           if (qt == 3) write_slot(4);
-          ok = round_with([&] {
+          ok = round_with([&](int who) {
+            if (who == 0) {                        // the dv accumulator
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_ts(tbase + kColDv, tbase + kColW + 8 * kk, adv(d_o_mn, 4096 * qt + 2048 * kk), id_wo,
-                     1u);
+              for (int kk = 0; kk < 2; ++kk)
+                mma_ts(tbase + kColDv, tbase + kColW + 8 * kk, adv(d_o_mn, 4096 * qt + 2048 * kk),
+                       id_wo, 1u);
+              if (qt == 3) issue_slots(4);
+            } else {                               // the dk accumulator
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-              mma_ts(tbase + kColDk, tbase + kColW + 16 + 8 * kk, adv(d_q_mn, 2048 * qt + 1024 * kk),
-                     id_mq, (qt > 0 || kk > 0) ? 1u : 0u);
-            if (qt == 3) issue_slots(4);
+              for (int kk = 0; kk < 2; ++kk)
+                mma_ts(tbase + kColDk, tbase + kColW + 16 + 8 * kk, adv(d_q_mn, 2048 * qt + 1024 * kk),
+                       id_mq, (qt > 0 || kk > 0) ? 1u : 0u);
+            }
           }, [&] {
             if (qt < 3) write_slot(qt + 1);
           });
@@ -1086,18 +1103,20 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         } else {
           rotate_left(R2, 4);
         }
-        auto issue_upd = [&] {
+        auto issue_upd = [&](int who) {
           const int ma = u < 2 ? u : 4, mb = 2 + u;
+          if (who == 0) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + kColR + 64 * ma, adv(d_tile, 2048 * kk), adv(d_o_mn, 2048 * kk), id_up, 1);
-          if (u < 2) {
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tbase + kColR + 64 * ma, adv(d_tile, 2048 * kk), adv(d_o_mn, 2048 * kk), id_up, 1);
+          }
+          if (u < 2 && who == 1) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tbase + kColR + 64 * mb, adv(d_tile, 32768 + 2048 * kk), adv(d_o_mn, 2048 * kk),
                      id_up, 1);
           }
-          if (u == 0) {
+          if (u == 0 && who == 0) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               mma_ss(tbase + kColRq, adv(d_cq, 1024 * kk), adv(d_q_mn, 1024 * kk), id_rq, 1);
