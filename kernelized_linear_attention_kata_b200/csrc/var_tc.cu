@@ -29,9 +29,10 @@
 // or leaves the kernel.
 //
 // Synchronous structure: 256 threads (two warps per TMEM lane quarter; half
-// h = warp / 4 splits the columns of each phase), thread 0 issues each round
-// of MMAs and commits it to one barrier every thread waits on. Independent
-// MMAs share rounds: per chunk
+// h = warp / 4 splits the columns of each phase), threads 0 and 32 issue
+// each round of MMAs (each accumulator's chain from one of them) and commit
+// it to one barrier every thread waits on. Independent MMAs share rounds:
+// per chunk
 //   1: U = Q Zd and the blocks of keys 0..63
 //   2: P V (keys 0..63, P in U's columns), the blocks of keys 64..127,
 //      readout groups 0, 1
@@ -235,7 +236,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
   if (threadIdx.x == 0) {
     mbar_init(&bars[kVBarLoadQ], 1);
     mbar_init(&bars[kVBarLoadKV], 1);
-    mbar_init(&bars[kVBarMma], 1);
+    mbar_init(&bars[kVBarMma], 2);                // one commit per issuing thread
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -274,9 +275,9 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 || threadIdx.x == 32) {    // issue(0), issue(1): one accumulator each
       tc_fence_after();
-      issue();
+      issue(threadIdx.x >> 5);
       mma_commit(&bars[kVBarMma]);
     }
     const bool ok = mbar_wait(&bars[kVBarMma], mph, abort_flag);
@@ -463,9 +464,12 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
         } else {
           tile_groups(IC<M0>{}, buf);
         }
-        return round([&] {
-          issue_update(M0, 0, M0 == 0);
-          if constexpr (M0 + 1 < NT) issue_update(M0 + 1, 1, false);
+        return round([&](int who) {
+          if (who == 0) {
+            issue_update(M0, 0, M0 == 0);
+          } else {
+            if constexpr (M0 + 1 < NT) issue_update(M0 + 1, 1, false);
+          }
         });
       };
       ok = update_round(IC<0>{});
@@ -547,11 +551,14 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
       static_assert(V != kMg2 || SH::ColW + 160 <= kVTmemCols, "P of the second key half");
 
       // round 1: U = Q Zd, the blocks of keys 0..63
-      ok = round([&] {
+      ok = round([&](int who) {
+        if (who == 0) {
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk)
-          mma_ss(tbase + SH::ColU, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_n32, kk);
-        issue_intra(0);
+          for (int kk = 0; kk < 2; ++kk)
+            mma_ss(tbase + SH::ColU, adv(d_q, 32 * kk), adv(d_z, 32 * kk), id_n32, kk);
+        } else {
+          issue_intra(0);
+        }
       });
       if (!ok) break;
       float den_inter = 0.f;
@@ -574,11 +581,14 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
       }
       if (half) slot_group(IC<1>{}); else slot_group(IC<0>{});
       // round 2: P V (keys 0..63), the blocks of keys 64..127, readout groups 0, 1
-      ok = round([&] {
-        issue_pv(0, SH::ColU);
-        issue_intra(1);
-        issue_readout(0);
-        issue_readout(1);
+      ok = round([&](int who) {
+        if (who == 0) {                          // the O accumulator
+          issue_pv(0, SH::ColU);
+          issue_readout(0);
+          issue_readout(1);
+        } else {
+          issue_intra(1);
+        }
       });
       if (!ok) break;
       {
@@ -593,13 +603,14 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
         if (half) tile_groups(IC<1>{}, buf + 32768); else tile_groups(IC<0>{}, buf);
       }
       // round 3: P V (keys 64..127), readout groups 2, 3, update of tiles 0, 1 and Z
-      ok = round([&] {
-        issue_pv(1, kColP1);
-        issue_readout(2);
-        if (NG > 4) issue_readout(3);
-        if (upd) {
+      ok = round([&](int who) {
+        if (who == 0) {                          // O, and state tile 1
+          issue_pv(1, kColP1);
+          issue_readout(2);
+          if (NG > 4) issue_readout(3);
+          if (upd) issue_update(1, 1, false);
+        } else if (upd) {                        // state tile 0 and Z
           issue_update(0, 0, true);
-          issue_update(1, 1, false);
         }
       });
       if (!ok) break;
@@ -607,9 +618,12 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
         // round 4 (Mg2): readout group 4, update of tile 2
         if (!half) slot_group(IC<4>{});
         if (upd && !half) tile_groups(IC<2>{}, buf);
-        ok = round([&] {
-          issue_readout(4);
-          if (upd) issue_update(2, 0, false);
+        ok = round([&](int who) {
+          if (who == 0) {
+            issue_readout(4);
+          } else if (upd) {
+            issue_update(2, 0, false);
+          }
         });
         if (!ok) break;
       }
