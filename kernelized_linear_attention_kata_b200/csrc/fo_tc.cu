@@ -20,13 +20,16 @@
 // segment's increment of S', the second gives segment g the sum of the
 // increments of segments 0 .. g-1 as its carry-in.
 //
-// Warp roles (320 threads): warp 0 TMA (Q, K, V, three stages each); warp 1
-// TMEM allocation and every MMA; warps 2-5 the query side (P); warps 6-9 the
-// state side (the bf16 snapshot of S' after each update, the epilogue and
-// the TMA store of y, the carry-in, the state written out). Per tile the
-// MMA warp issues the update before the readout, so the snapshot of S'_i+1
-// (double-buffered) is taken while the readout of tile i runs. Math thread r owns
-// TMEM lane r: token r of the tile, or feature row r of S'.
+// Warp roles (352 threads): warp 0 TMA (Q, K, V, three stages each); warp 1
+// TMEM allocation and the MMAs of Q K^T, P V and the readout (in the
+// increment kernel, the update); warp 10 the update of S' in the pass (one
+// thread issues an MMA only every ~80 cycles, so the two streams go
+// side by side); warps 2-5 the query side (P); warps 6-9 the state side (the
+// bf16 snapshot of S' after each update, the epilogue and the TMA store of
+// y, the carry-in, the state written out). The readout of tile i reads the
+// snapshot of S'_i, so the snapshot of S'_i+1 (double-buffered) is taken
+// while it runs. Math thread r owns TMEM lane r: token r of the tile, or
+// feature row r of S'.
 //
 // Tensor memory (512 columns): S' [0, 80) (lanes 0..64 used), O' [128, 208),
 // Q K^T of even / odd tiles [256, 384) / [384, 512) (P in place as bf16).
@@ -45,7 +48,7 @@ constexpr int kTile = 128;         // tokens per tile
 constexpr int kDh = 64;            // d_k = d_v
 constexpr int kNa = 80;            // augmented width (65 padded to a multiple of 16)
 constexpr int kRows = 65;          // rows / columns of S' that carry data
-constexpr int kThreads = 320;      // 10 warps
+constexpr int kThreads = 352;      // 11 warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 128, kColX = 256;   // X of tile i at kColX + 128 (i & 1)
 constexpr int kAggFloats = kRows * kRows;                 // one segment increment: S'[0..64][0..64]
@@ -157,14 +160,14 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
       mbar_init(&bars[kBarQFull + s], 1);
       mbar_init(&bars[kBarQEmpty + s], 1);
       mbar_init(&bars[kBarKvFull + s], 1);
-      mbar_init(&bars[kBarKvEmpty + s], 1);
+      mbar_init(&bars[kBarKvEmpty + s], AGG ? 1 : 2);     // pass: both issuing warps
     }
     for (int s = 0; s < 2; ++s) mbar_init(&bars[kBarSFull + s], 1);
     mbar_init(&bars[kBarPFull], A);
     mbar_init(&bars[kBarOFull], 1);
     mbar_init(&bars[kBarOFree], A);
     mbar_init(&bars[kBarSnapFull], A);
-    mbar_init(&bars[kBarSnapFree], 1);
+    mbar_init(&bars[kBarSnapFree], 2);              // both issuing warps
     mbar_init(&bars[kBarStageFull], A);
     mbar_init(&bars[kBarStageFree], 1);
     mbar_init(&bars[kBarUpdFull], 1);
@@ -260,14 +263,9 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tbase + kColO, x + 8 * kk, adv(d_v1[st], 2048 * kk), id_pv, kk);
-          // S' += [K | 1]^T [V | 1] first: the readout below reads the
-          // snapshot of S'_i (in shared memory), so the state side can take
-          // the snapshot of S'_i+1 while the readout runs
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tbase + kColS, adv(d_k1[st], 2048 * kk), adv(d_v1[st], 2048 * kk), id_up, 1);
-          // S' updated; also tile i - 1's readout (issued before) has read
-          // the other snapshot buffer
+          // tile i - 1's readout (issued before) has read the other snapshot
+          // buffer; K_i (Q K^T) and V_i (P V) are read. Warp 10 adds its
+          // commits for the update of S'.
           mma_commit(&bars[kBarSnapFree]);
           mma_commit(&bars[kBarKvEmpty + st]);
           // O' += [Q | 1] S'_i
@@ -278,8 +276,34 @@ fo_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CU
           mma_commit(&bars[kBarOFull]);
           mma_commit(&bars[kBarQEmpty + st]);
         }
-        if (ok && ntiles > 0) mma_commit(&bars[kBarUpdFull]);
       }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------ MMA issue: the update
+    // S' += [K | 1]^T [V | 1], issued beside warp 1's stream (one thread
+    // issues an MMA only every ~80 cycles). The readout of tile i reads the
+    // snapshot of S'_i in shared memory, so the state side takes the snapshot
+    // of S'_i+1 while it runs.
+    if (!AGG && lane == 0) {
+      constexpr uint32_t id_up = idesc_bf16(128, kNa, true, true);
+      auto adv = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+      const uint32_t a_k = smem_u32(smem + L::kOffK), a_v = smem_u32(smem + L::kOffV);
+      const uint32_t a_ones = smem_u32(smem + L::kOffOnes);
+      bool ok = true;
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int st = i % kStages;
+        const uint64_t d_v1 = smem_desc(a_v + 16384 * st, a_ones - (a_v + 16384 * st), 1024, kSw128);
+        const uint64_t d_k1 = smem_desc(a_k + 16384 * st, a_ones - (a_k + 16384 * st), 1024, kSw128);
+        // PFull(i): the snapshot of S'_i is taken and tile i's K, V are loaded
+        if (!(ok = mbar_wait(&bars[kBarPFull], i & 1, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tbase + kColS, adv(d_k1, 2048 * kk), adv(d_v1, 2048 * kk), id_up, 1);
+        mma_commit(&bars[kBarSnapFree]);
+        mma_commit(&bars[kBarKvEmpty + st]);
+      }
+      if (ok && ntiles > 0) mma_commit(&bars[kBarUpdFull]);
     }
   } else if (warp < 6) {
     // ------------------------------------------------ query side (warps 2..5)
