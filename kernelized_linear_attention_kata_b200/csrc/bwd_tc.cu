@@ -56,6 +56,8 @@ namespace {
 using namespace tc;
 using namespace psd;
 
+template <int N> using IC = std::integral_constant<int, N>;
+
 constexpr int kBThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColZ = 320, kColDq = 352, kColA = 384, kColB = 448;
@@ -448,11 +450,58 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
         for (int l = 0; l < 32; ++l) dqc[l] = inv * (h[l] + row[l]) + 2.f * ct * u[l];
       }
     };
+    // The update S += phi(K)^T V, Z += K^T K (the state of the next chunk)
+    // rides in the next three rounds, which touch neither S nor Z: update
+    // round U (tiles (0, 2) and Z, then (1, 3), then 4) in the combine round,
+    // the first dq += M K round and the second intra round. Its key features
+    // (two 32 KB tiles, one per half) are written before each of them.
+    const bool upd = i + 1 < nchunks;        // the state after the segment is not needed
+    auto write_upd = [&](auto uc) {
+      constexpr int U = decltype(uc)::value;
+      constexpr int M0 = U < 2 ? U : 4, M1 = U < 2 ? 2 + U : -1;   // this round's tiles, per half
+      uint32_t XK[16], P[32], R2[32];
+      load_pairs(smem + L::K, r, XK, P);
+      if (!half) {
+#pragma unroll
+        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[(l + 4 * M0) & 31], 0x40004000u);   // x 2.0
+        write_tile(smem + L::Key, r, M0 == kTiles - 1, M0 == 0 ? 0x3f003f00u : 0x3f803f80u, P, R2);
+      } else if constexpr (M1 >= 0) {
+#pragma unroll
+        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[(l + 4 * M1) & 31], 0x40004000u);
+        write_tile(smem + L::Key + 32768, r, false, 0x3f803f80u, P, R2);
+      }
+    };
+    auto issue_upd = [&](int u, int who) {
+      const int ma = u < 2 ? u : 4, mb = 2 + u;
+      if (who == 0) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tbase + kColS + 64 * ma, adv(d_key, 2048 * kk), adv(d_v_mn, 2048 * kk), id_up, 1);
+        if (u == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tbase + kColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1);
+        }
+      } else if (u < 2) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tbase + kColS + 64 * mb, adv(d_key, 32768 + 2048 * kk), adv(d_v_mn, 2048 * kk),
+                 id_up, 1);
+      }
+    };
     for (int b = 0; ok && b < 2; ++b) {
       if (b == 0) {
-        ok = round_with([&](int who) { issue_intra(0, who); }, combine);
+        if (upd) write_upd(IC<0>{});
+        ok = round_with([&](int who) {
+          issue_intra(0, who);
+          if (upd) issue_upd(0, who);
+        }, combine);
       } else {
-        ok = round([&](int who) { issue_intra(1, who); });
+        if (upd) write_upd(IC<2>{});
+        ok = round([&](int who) {
+          issue_intra(1, who);
+          if (upd) issue_upd(2, who);
+        });
       }
       if (!ok) break;
       if (b == 1 && threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);   // Q, dout read
@@ -471,14 +520,17 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
         const float m1 = s0 + 2 * j + 1 <= r ? 2.f * a1 * e1 : 0.f;
         m[j] = pack_bf16x2(m0, m1);
       }
+      if (b == 0 && upd) write_upd(IC<1>{});   // update round 0 (the last round) read its tiles
       __syncthreads();          // every thread has read A and D' before M overwrites A
       tmem_st16(tbase + lane_off + kColA + 16 * half, m);
       ok = round([&](int who) {
-        if (who != 0) return;                    // one accumulator: one issuing thread
+        if (who == 0) {                          // one accumulator: one issuing thread
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tbase + kColDq, tbase + kColA + 8 * kk, adv(d_k_mn, 4096 * b + 1024 * kk), id_mk,
-                 (b > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tbase + kColDq, tbase + kColA + 8 * kk, adv(d_k_mn, 4096 * b + 1024 * kk), id_mk,
+                   (b > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (b == 0 && upd) issue_upd(1, who);
       });
     }
     if (!ok) break;
@@ -505,48 +557,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
     write_dq();
     if (i == nchunks - 1) break;            // the state after the segment is not needed
 
-    // ---- update: S += phi(K)^T V, Z += K^T K; three rounds of two key tiles ----
-    {
-      uint32_t XK[16], P[32], R2[32];
-      load_pairs(smem + L::K, r, XK, P);
-#pragma unroll
-      for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[l], 0x40004000u);   // x 2.0
-      // tiles: round 0 (0, 2), round 1 (1, 3), round 2 (4, -)
-      if (half) rotate_left(R2, 8);
-      for (int u = 0; ok && u < 3; ++u) {
-        const int m = half ? (u < 2 ? 2 + u : -1) : (u < 2 ? u : 4);
-        if (m >= 0)
-          write_tile(smem + L::Key + 32768 * half, r, m == kTiles - 1,
-                     m == 0 ? 0x3f003f00u : 0x3f803f80u, P, R2);
-        if (!half && u == 1) {
-          rotate_left(R2, 12);
-        } else {
-          rotate_left(R2, 4);
-        }
-        auto issue_upd = [&](int who) {
-          const int ma = u < 2 ? u : 4, mb = 2 + u;
-          if (who == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tbase + kColS + 64 * ma, adv(d_key, 2048 * kk), adv(d_v_mn, 2048 * kk), id_up, 1);
-          }
-          if (u < 2 && who == 1) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tbase + kColS + 64 * mb, adv(d_key, 32768 + 2048 * kk), adv(d_v_mn, 2048 * kk),
-                     id_up, 1);
-          }
-          if (u == 0 && who == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tbase + kColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1);
-          }
-        };
-        ok = round(issue_upd);
-      }
-      if (!ok) break;
-      if (threadIdx.x == 0) load_kv(i + 1);           // K, V of this chunk no longer read
-    }
+    if (threadIdx.x == 0) load_kv(i + 1);             // K, V of this chunk no longer read
     // ---- snapshot S_c+1 (half 0: tiles 0, 1, 4; half 1: tiles 2, 3) and Z_c+1 ----
     for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
       const int mt = (!half && m == 2) ? 4 : m;
