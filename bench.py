@@ -139,7 +139,7 @@ KERNEL_SOURCES = {
     "tc_fo_increment": ["fo_tc.cu", "tc_common.cuh", "common.cuh"],
     "tc_bwd_dq": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
     "tc_bwd_dkdv": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
-    "tc_bwd_suffix_increment": ["bwd_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
+    "tc_bwd_suffix_increment": ["chunked_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
     "tc_variant_pass": ["var_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
     "tc_variant_increment": ["var_tc.cu", "psd_tc_common.cuh", "tc_common.cuh", "common.cuh"],
 }

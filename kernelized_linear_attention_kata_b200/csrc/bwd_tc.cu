@@ -610,8 +610,9 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
 //   [384, 448)  the dv accumulator (first a 64-feature Y block of half 0)
 //   [448, 512)  work: a Y block of half 1; K Q^T | V dout^T (32 queries
 //               each); W~ | M (bf16)
-// The increment kernel (AGG) runs only the update over its segment and
-// writes the segment's (R', Rq) increment.
+// The suffix increments (R', Rq of segments 1 .. G-1, the carry-in of the
+// earlier segments) come from the forward's increment kernel in its suffix
+// form (psd_tc_suffix_increments).
 // ---------------------------------------------------------------------------
 constexpr uint32_t kColR = 0, kColRq = 320, kColDk = 352, kColDv = 384, kColW = 448;
 constexpr int kQSlotsPsd = 9;      // 64-feature slots of the readout (the last holds 16)
@@ -640,7 +641,6 @@ struct DkvSmem {
   static_assert(Bytes <= 232448, "shared memory budget");
 };
 
-template <bool AGG>
 __global__ void __launch_bounds__(kBThreads, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
@@ -667,13 +667,11 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
   const int quarter = warp & 3, half = warp >> 2;
   const int r = quarter * 32 + lane;
   const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-  // the increment kernel covers segments 1 .. G-1 (the carry of the earlier ones)
-  const int G_grid = AGG ? G - 1 : G;
-  const int g = blockIdx.x % G_grid + (AGG ? 1 : 0), bh = blockIdx.x / G_grid;
+  const int g = blockIdx.x % G, bh = blockIdx.x / G;
   const int t0 = g * seg_len, t1 = min(T, t0 + seg_len);
   const int nchunks = (t1 - t0 + kC - 1) / kC;
-  // chunk order: the pass walks backwards, the increment kernel forwards
-  auto chunk_of = [&](int i) { return AGG ? i : nchunks - 1 - i; };
+  // the pass walks its chunks backwards
+  auto chunk_of = [&](int i) { return nchunks - 1 - i; };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kBarLoadQ], 1);
@@ -707,11 +705,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     tma_prefetch_desc(&tmq);
     tma_prefetch_desc(&tmo);
     load_q(0);
-    if (!AGG) {
-      tma_prefetch_desc(&tmk);
-      tma_prefetch_desc(&tmv);
-      load_kv(0);
-    }
+    tma_prefetch_desc(&tmk);
+    tma_prefetch_desc(&tmv);
+    load_kv(0);
   }
 
   uint32_t mph = 0;
@@ -761,8 +757,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
   constexpr uint32_t id_up = idesc_bf16(128, 64, true, true);
   constexpr uint32_t id_rq = idesc_bf16(128, 32, true, true);
 
-  // ---- carry-in: R', Rq = the increments of segments g+1 .. G-1 (zero in
-  //      the increment kernel) ----
+  // ---- carry-in: R', Rq = the increments of segments g+1 .. G-1 ----
   {
     const float *seg0 = aggR + (size_t)bh * G * kAggFloats;
     for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
@@ -773,7 +768,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
         float acc[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) acc[c] = 0.f;
-        if (!AGG && f < kD) {
+        if (f < kD) {
           for (int gp = g + 1; gp < G; ++gp) {
             const float4 *src =
                 reinterpret_cast<const float4 *>(seg0 + (size_t)gp * kAggFloats + f * kDV + 16 * q4);
@@ -791,7 +786,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
 #pragma unroll
         for (int c = 0; c < 16; ++c) bits[c] = __float_as_uint(acc[c]);
         tmem_st16(tbase + lane_off + kColR + 64 * mt + 16 * q4, bits);
-        if (!AGG && f < kD) {
+        if (f < kD) {
           *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4)) = pack8(bits);
           *reinterpret_cast<uint4 *>(snap + sw128(f, 2 * q4 + 1)) = pack8(bits + 8);
         }
@@ -801,7 +796,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
       float acc[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) acc[c] = 0.f;
-      if (!AGG && r < kDK) {
+      if (r < kDK) {
         for (int gp = g + 1; gp < G; ++gp) {
           const float4 *src =
               reinterpret_cast<const float4 *>(seg0 + (size_t)gp * kAggFloats + kD * kDV + r * kDK);
@@ -819,7 +814,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
 #pragma unroll
       for (int c = 0; c < 32; ++c) bits[c] = __float_as_uint(acc[c]);
       tmem_st32(tbase + lane_off + kColRq, bits);
-      if (!AGG && quarter == 0) {
+      if (quarter == 0) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4 *>(rqsnap + sw64(r, c)) = pack8(bits + 8 * c);
       }
@@ -847,7 +842,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     const bool valid = c0 + r < T;
     // dk = the intra part + the carried part from ubuf (half 0); dv (half 1)
     auto write_outputs = [&] {
-      if constexpr (!AGG) {
+      {
         if (!half) {
           uint32_t acc[32];
           tmem_ld32(tbase + lane_off + kColDk, acc);
@@ -889,7 +884,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     }
     if (i + 1 < nchunks) fetch_dc(i + 1);
     __syncthreads();
-    if (!AGG) {
+    {
       if (!(ok = wait_all(&bars[kBarLoadKV], i & 1))) break;
       float kf[32];
       row_f32(smem + L::K, r, kf);
@@ -1079,7 +1074,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
       if (!ok) break;
       if (threadIdx.x == 0 && i + 1 < nchunks) load_kv(i + 1);    // K, V no longer read
     }
-    if (!AGG && i == nchunks - 1) {            // the state before the segment is not needed
+    if (i == nchunks - 1) {                    // the state before the segment is not needed
       write_outputs();
       break;
     }
@@ -1140,7 +1135,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
       if (threadIdx.x == 0 && i + 1 < nchunks) load_q(i + 1);     // Q, dout no longer read
     }
     // ---- snapshot R' (half 0: tiles 0, 1, 4; half 1: tiles 2, 3) and Rq ----
-    if constexpr (!AGG) {
+    {
     for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
       const int mt = (!half && m == 2) ? 4 : m;
       if (mt == 4 && quarter != 0) continue;
@@ -1167,39 +1162,6 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
     }
   }
 
-  // ---- the increment kernel writes its segment's (R', Rq) ----
-  if (AGG && ok && nchunks > 0) {
-    float *dst = aggR + ((size_t)bh * G + g) * kAggFloats;
-    for (int m = half ? 2 : 0; m < (half ? 4 : 3); ++m) {
-      const int mt = (!half && m == 2) ? 4 : m;
-      if (mt == 4 && quarter != 0) continue;
-      const int f = 128 * mt + r;
-      uint32_t a[32], b2[32];
-      tmem_ld32(tbase + lane_off + kColR + 64 * mt, a);
-      tmem_ld32(tbase + lane_off + kColR + 64 * mt + 32, b2);
-      tmem_wait_ld();
-      if (f < kD) {
-        float4 *row = reinterpret_cast<float4 *>(dst + (size_t)f * kDV);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          row[c] = make_float4(__uint_as_float(a[4 * c]), __uint_as_float(a[4 * c + 1]),
-                               __uint_as_float(a[4 * c + 2]), __uint_as_float(a[4 * c + 3]));
-          row[8 + c] = make_float4(__uint_as_float(b2[4 * c]), __uint_as_float(b2[4 * c + 1]),
-                                   __uint_as_float(b2[4 * c + 2]), __uint_as_float(b2[4 * c + 3]));
-        }
-      }
-    }
-    if (half && quarter == 0) {
-      uint32_t zr[32];
-      tmem_ld32(tbase + lane_off + kColRq, zr);
-      tmem_wait_ld();
-      float4 *row = reinterpret_cast<float4 *>(dst + kD * kDV + r * kDK);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        row[c] = make_float4(__uint_as_float(zr[4 * c]), __uint_as_float(zr[4 * c + 1]),
-                             __uint_as_float(zr[4 * c + 2]), __uint_as_float(zr[4 * c + 3]));
-    }
-  }
   if (*abort_flag && threadIdx.x == 0) flag_status(status, kStatusDeviceTimeout);
   tc_fence_before();
   __syncthreads();
@@ -1237,16 +1199,13 @@ cudaError_t tc_bwd_dkdv(const BackwardLaunch &a, float *aggR, int G, int seg_len
       !make_tma_3d_bf16(&to, a.dout, kDV, a.T, a.BH, kC))
     return cudaErrorInvalidValue;
   cudaError_t e;
-  if (G > 1) {
-    auto kinc = bwd_dkdv_tc_kernel<true>;
-    e = cudaFuncSetAttribute(kinc, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvSmem::Bytes);
-    if (e != cudaSuccess) return e;
-    ProfileScope prof("tc_bwd_suffix_increment", a.stream);
-    kinc<<<(unsigned)(a.BH * (G - 1)), kBThreads, DkvSmem::Bytes, a.stream>>>(
-        tq, tk, tv, to, aggR, a.den, a.c, nullptr, nullptr, a.status, a.T, G, seg_len);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  auto kern = bwd_dkdv_tc_kernel<false>;
+  // the suffix increments of segments 1 .. G-1 run on the forward's
+  // warp-specialised increment kernel (K := Q, V := dout, scaled by 1 / d_t,
+  // K^T K weighted by c_t)
+  if ((e = psd_tc_suffix_increments(a.q, a.dout, a.den, a.c, aggR, a.status, a.BH, a.T, G, seg_len,
+                                    a.stream)) != cudaSuccess)
+    return e;
+  auto kern = bwd_dkdv_tc_kernel;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DkvSmem::Bytes);
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_bwd_dkdv", a.stream);

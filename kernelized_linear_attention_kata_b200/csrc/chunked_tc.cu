@@ -94,11 +94,12 @@ __host__ __device__ constexpr uint32_t ring_col(int e) { return e == 3 ? kColU :
 // 64 features, K-major) and three tensor-memory slots.
 constexpr int kKSlotBytes = 32768;
 constexpr int kQSlots = 9;          // 64-feature readout slots per chunk
-template <bool AGG>
+template <bool AGG, bool SFX = false>
 struct Layout {
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = AGG ? 0 : 8192;
-  static constexpr int kOffV = kOffK + 16384;
+  static constexpr int kOffCQ = kOffK + 16384;        // suffix increments: c_t q_t, two stages
+  static constexpr int kOffV = kOffCQ + (SFX ? 16384 : 0);
   static constexpr int kOffSnap = kOffV + 32768;      // [528][64] bf16, 128 B rows (pass only)
   static constexpr int kOffZSnap = kOffSnap + (AGG ? 0 : kD * 128);   // [32][32] bf16, 64 B rows
   static constexpr int kOffStage = kOffZSnap + (AGG ? 0 : 2048);      // y: [128][64] bf16, 128 B rows
@@ -122,14 +123,28 @@ enum {
 constexpr int kBarBytes = 8 * kNumBars;
 static_assert(kBarBytes + 8 <= 1024, "barrier area");
 
-template <bool AGG>
+// 2 / d_t of token t as a bf16 pair (0 past T or for d_t = 0): the suffix
+// increments' scale of the query features.
+__device__ __forceinline__ uint32_t suffix_scale(const float *den, int bh, int T, int t) {
+  const float d = t < T ? den[(size_t)bh * T + t] : 0.f;
+  const float s = d != 0.f ? 2.f / d : 0.f;
+  return tc::pack_bf16x2(s, s);
+}
+
+// SFX (with AGG): the backward's suffix increments of segments g_off ..
+// g_off + G_grid - 1, with K := Q, V := dout, the key features scaled by
+// 2 / d_t instead of 2 and K^T K weighted by c_t: R' = sum m_f phi(q_t)
+// dout_t^T / d_t, Rq = Q^T diag(c) Q (tok_den, tok_c: [BH][T]).
+template <bool AGG, bool SFX = false>
 __global__ void __launch_bounds__(kThreads, 1)
 chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
                   float *__restrict__ agg, const float *__restrict__ S0, const float *__restrict__ z0,
                   float *__restrict__ S_out, float *__restrict__ z_out,
-                  unsigned *__restrict__ status, int T, int G_grid, int G_total, int seg_len) {
-  using L = Layout<AGG>;
+                  unsigned *__restrict__ status, int T, int G_grid, int G_total, int seg_len,
+                  const float *__restrict__ tok_den, const float *__restrict__ tok_c, int g_off) {
+  static_assert(AGG || !SFX, "the suffix form is an increment kernel");
+  using L = Layout<AGG, SFX>;
   constexpr int NK = L::kKRingSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -140,7 +155,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int g = blockIdx.x % G_grid;
+  const int g = blockIdx.x % G_grid + g_off;
   const int bh = blockIdx.x / G_grid;
   const int t0 = g * seg_len;
   const int t1 = min(T, t0 + seg_len);
@@ -252,6 +267,8 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
       const uint64_t d_kring = smem_desc(kring_a, 16384, 1024, kSw128);         // update A
       const uint64_t d_k_k = smem_desc(smem_u32(smem + L::kOffK), 16, 512, kSw64);     // K, K-major
       const uint64_t d_k_mn = smem_desc(smem_u32(smem + L::kOffK), 8192, 512, kSw64);  // K, MN-major
+      // c_t q_t (suffix increments), MN-major: the weighted K^T K's A operand
+      const uint64_t d_cq_mn = smem_desc(smem_u32(smem + L::kOffCQ), 8192, 512, kSw64);
       const uint64_t d_v = smem_desc(smem_u32(smem + L::kOffV), 16384, 1024, kSw128);  // V, MN-major
       // Key-ring slots are shared memory written by threads (ordered for the
       // tensor core by their proxy fence and the mbarrier), so their waits
@@ -369,7 +386,7 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
               // Z += K^T K (A rows 32..127 alias other shared memory; unused lanes)
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tbase + kColZ, adv(d_k_mn, 8192 * st + 1024 * kk),
+                mma_ss(tbase + kColZ, adv(SFX ? d_cq_mn : d_k_mn, 8192 * st + 1024 * kk),
                        adv(d_k_mn, 8192 * st + 1024 * kk), id_z, 1);
               if (!AGG) mma_commit(&bars[kBarZDone]);
             }
@@ -561,9 +578,22 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         if (!(ok = warp_wait(&bars[kBarKvFull + st], (i >> 1) & 1, abort_flag))) break;
         uint32_t XK[16], P[32], R2[32];
         load_pairs(smem + L::kOffK + 8192 * st, r, XK, P);
+        const uint32_t sc2 = SFX ? suffix_scale(tok_den, bh, T, t0 + i * kC + r) : 0x40004000u;
+        if constexpr (SFX) {
+          // c_t q_t for the weighted K^T K (read by warp 1 after this set's tile 1)
+          const int t = t0 + i * kC + r;
+          const float c = t < T ? tok_c[(size_t)bh * T + t] : 0.f;
+          const uint32_t cc2 = tc::pack_bf16x2(c, c);
+          uint8_t *cq = smem + L::kOffCQ + 8192 * st;
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            *reinterpret_cast<uint4 *>(cq + sw64(r, c4)) =
+                make_uint4(bmul2(XK[4 * c4], cc2), bmul2(XK[4 * c4 + 1], cc2), bmul2(XK[4 * c4 + 2], cc2),
+                           bmul2(XK[4 * c4 + 3], cc2));
+        }
         warp_arrive(&bars[kBarKvEmpty + st]);           // K rows read
 #pragma unroll
-        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[(l + 4) & 31], 0x40004000u);   // x 2, rotated by 4
+        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[(l + 4) & 31], sc2);   // x 2 (or 2 / d_t), rotated by 4
 #pragma unroll 1
         for (int m = 1; m < kTiles; m += 2) {
           const int u = i * kTiles + m;
@@ -678,8 +708,9 @@ chunked_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         uint32_t XK[16], P[32], R2[32];
         load_pairs(smem + L::kOffK + 8192 * st, r, XK, P);
         warp_arrive(&bars[kBarKvEmpty + st]);         // K rows read
+        const uint32_t sc2 = SFX ? suffix_scale(tok_den, bh, T, t0 + i * kC + r) : 0x40004000u;
 #pragma unroll
-        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[l], 0x40004000u);   // x 2.0
+        for (int l = 0; l < 32; ++l) R2[l] = bmul2(P[l], sc2);   // x 2.0 (suffix: x 2 / d_t)
 #pragma unroll 1
         for (int m = 0; m < kTiles; ++m) {
           const int u = i * kTiles + m;
@@ -831,7 +862,8 @@ cudaError_t launch_increments(const CUtensorMap &tq, const CUtensorMap &tk, cons
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_segment_increment", stream);
   kagg<<<(unsigned)(BH * G_inc), kThreads, Layout<true>::kSmemBytes, stream>>>(
-      tq, tk, tv, to, agg, nullptr, nullptr, nullptr, nullptr, status, T, G_inc, G_total, seg_len);
+      tq, tk, tv, to, agg, nullptr, nullptr, nullptr, nullptr, status, T, G_inc, G_total, seg_len,
+      nullptr, nullptr, 0);
   return cudaGetLastError();
 }
 }  // namespace
@@ -844,6 +876,25 @@ cudaError_t psd_tc_increments(const void *k, const void *v, float *agg, unsigned
   if (!make_tma_3d_bf16(&tk, k, kDK, T, BH, kC) || !make_tma_3d_bf16(&tv, v, kDV, T, BH, kC))
     return cudaErrorInvalidValue;
   return launch_increments(tk, tk, tv, tv, agg, status, BH, T, G_inc, G_total, seg_len, stream);
+}
+
+cudaError_t psd_tc_suffix_increments(const void *q, const void *dout, const float *den,
+                                     const float *c, float *aggR, unsigned *status, long long BH,
+                                     int T, int G, int seg_len, cudaStream_t stream) {
+  if (G <= 1) return cudaSuccess;
+  CUtensorMap tq, to;
+  if (!make_tma_3d_bf16(&tq, q, kDK, T, BH, kC) || !make_tma_3d_bf16(&to, dout, kDV, T, BH, kC))
+    return cudaErrorInvalidValue;
+  auto ksfx = chunked_tc_kernel<true, true>;
+  cudaError_t e = cudaFuncSetAttribute(ksfx, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Layout<true, true>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  ProfileScope prof("tc_bwd_suffix_increment", stream);
+  // segments 1 .. G-1 (the suffix carry of the earlier ones)
+  ksfx<<<(unsigned)(BH * (G - 1)), kThreads, Layout<true, true>::kSmemBytes, stream>>>(
+      tq, tq, to, to, aggR, nullptr, nullptr, nullptr, nullptr, status, T, G - 1, G, seg_len, den, c,
+      1);
+  return cudaGetLastError();
 }
 
 cudaError_t tc_chunked(const ChunkedLaunch &a) {
@@ -872,7 +923,8 @@ cudaError_t tc_chunked(const ChunkedLaunch &a) {
   if (e != cudaSuccess) return e;
   ProfileScope prof("tc_segment_pass", a.stream);
   kpass<<<(unsigned)(a.BH * G), kThreads, Layout<false>::kSmemBytes, a.stream>>>(
-      tq, tk, tv, to, a.agg, a.S0, a.z0, a.S_out, a.z_out, a.status, a.T, G, G, seg_len);
+      tq, tk, tv, to, a.agg, a.S0, a.z0, a.S_out, a.z_out, a.status, a.T, G, G, seg_len, nullptr,
+      nullptr, 0);
   return cudaGetLastError();
 }
 

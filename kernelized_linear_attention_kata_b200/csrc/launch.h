@@ -127,6 +127,12 @@ cudaError_t tc_bwd_dkdv(const BackwardLaunch &a, float *aggR, int G, int seg_len
 cudaError_t psd_tc_increments(const void *k, const void *v, float *agg, unsigned *status,
                               long long BH, int T, int G_inc, int G_total, int seg_len,
                               cudaStream_t stream);
+// The backward's suffix increments on the same kernel: segments 1 .. G-1,
+// R' = sum m_f phi(q_t) dout_t^T / d_t and Rq = Q^T diag(c) Q into aggR[bh][g]
+// (the increment layout), from d_t and c_t ([BH][T] fp32).
+cudaError_t psd_tc_suffix_increments(const void *q, const void *dout, const float *den,
+                                     const float *c, float *aggR, unsigned *status, long long BH,
+                                     int T, int G, int seg_len, cudaStream_t stream);
 // The PSD tensor-core forward's split: G segments of seg_len tokens per head,
 // each segment's increment computed as P pieces (G * P increments per head in
 // the workspace).
