@@ -94,7 +94,13 @@ struct VarSmem {
                 "swizzle atoms");
   static_assert(Bytes <= 232448, "shared memory budget");
 };
-enum { kVBarLoadQ = 0, kVBarLoadKV, kVBarMma, kVNumBars };
+enum { kVBarLoadQ = 0, kVBarLoadKV, kVBarLoadKV1, kVBarMma, kVNumBars };
+// The increment kernel double-buffers K, V: its second stage sits in the
+// snapshot area (unused there), kKvStage1 bytes above the first.
+constexpr int kKvStage1 = VarSmem::Snap - VarSmem::K;
+static_assert(VarSmem::K + kKvStage1 + 8192 <= VarSmem::V + kKvStage1 &&
+                  VarSmem::V + kKvStage1 + 16384 <= VarSmem::ZSnap && (VarSmem::V + kKvStage1) % 1024 == 0,
+              "second K, V stage inside the snapshot area");
 
 // Pairs of one 16-wide half h of a row: P[l] = (x_(16h+l), x_(16h+(l+1) mod 16)),
 // from the row's 16 bf16x2 words X.
@@ -236,6 +242,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
   if (threadIdx.x == 0) {
     mbar_init(&bars[kVBarLoadQ], 1);
     mbar_init(&bars[kVBarLoadKV], 1);
+    mbar_init(&bars[kVBarLoadKV1], 1);
     mbar_init(&bars[kVBarMma], 2);                // one commit per issuing thread
     *abort_flag = 0;
     mbar_init_fence();
@@ -253,10 +260,13 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     mbar_arrive_expect_tx(&bars[kVBarLoadQ], 8192);
     tma_load_3d(smem + L::Q, &tmq, &bars[kVBarLoadQ], 0, t0 + i * kVC, bh);
   };
+  // K and V of chunk i; the increment kernel alternates two stages
   auto load_kv = [&](int i) {
-    mbar_arrive_expect_tx(&bars[kVBarLoadKV], 8192 + 16384);
-    tma_load_3d(smem + L::K, &tmk, &bars[kVBarLoadKV], 0, t0 + i * kVC, bh);
-    tma_load_3d(smem + L::V, &tmv, &bars[kVBarLoadKV], 0, t0 + i * kVC, bh);
+    const int st = AGG ? (i & 1) : 0;
+    uint64_t *bar = &bars[kVBarLoadKV + st];
+    mbar_arrive_expect_tx(bar, 8192 + 16384);
+    tma_load_3d(smem + L::K + kKvStage1 * st, &tmk, bar, 0, t0 + i * kVC, bh);
+    tma_load_3d(smem + L::V + kKvStage1 * st, &tmv, bar, 0, t0 + i * kVC, bh);
   };
   if (threadIdx.x == 0 && nchunks > 0) {
     tma_prefetch_desc(&tmk);
@@ -266,6 +276,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
       load_q(0);
     }
     load_kv(0);
+    if (AGG && nchunks > 1) load_kv(1);
   }
 
   uint32_t mph = 0;
@@ -309,9 +320,12 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
   //      increments of the earlier segments; the snapshot's rows past D are
   //      zero (the last readout K-step reads 16 rows) ----
   {
-    for (int e = threadIdx.x; e < (384 - D) * 8; e += kVThreads)
-      *reinterpret_cast<uint4 *>(snap + (size_t)(D + e / 8) * 128 + (e % 8) * 16) =
-          make_uint4(0u, 0u, 0u, 0u);
+    // (the increment kernel has no readout, and holds its second K, V stage
+    // in the snapshot area)
+    if (!AGG)
+      for (int e = threadIdx.x; e < (384 - D) * 8; e += kVThreads)
+        *reinterpret_cast<uint4 *>(snap + (size_t)(D + e / 8) * 128 + (e % 8) * 16) =
+            make_uint4(0u, 0u, 0u, 0u);
     const float *seg0 = agg + (size_t)bh * G_total * kInc;
     for (int mt = half; mt < NT; mt += 2) {
       const int f = 128 * mt + r;
@@ -425,12 +439,14 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
   for (int i = 0; ok && i < nchunks; ++i) {
     const int c0 = t0 + i * kVC;
     const bool valid = c0 + r < T;
-    if (!(ok = wait_all(&bars[kVBarLoadKV], i & 1))) break;
+    const int kvs = AGG ? (i & 1) : 0;                  // K, V stage of this chunk
+    const uint32_t kvo = (uint32_t)(kKvStage1 * kvs);
+    if (!(ok = wait_all(&bars[kVBarLoadKV + kvs], AGG ? (i >> 1) & 1 : i & 1))) break;
     // key tile M of the update (groups 2 M, 2 M + 1) into tile buffer tb
     auto tile_groups = [&](auto mc, uint8_t *tb) {
       constexpr int M = decltype(mc)::value;
       uint32_t XK[16], Ka[16], Kb[16], w[32];
-      row_words(smem + L::K, r, XK);
+      row_words(smem + L::K + kvo, r, XK);
       half_pairs(XK, 0, Ka);
       half_pairs(XK, 1, Kb);
       if constexpr (2 * M < NG) {
@@ -446,12 +462,12 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
     auto issue_update = [&](int M, int hb, bool with_z) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_ss(tbase + SH::ColS + 64 * M, adv(d_tile, 32768 * hb + 2048 * kk), adv(d_v_mn, 2048 * kk),
-               id_up, 1u);
+        mma_ss(tbase + SH::ColS + 64 * M, adv(d_tile, 32768 * hb + 2048 * kk),
+               adv(d_v_mn, kvo + 2048 * kk), id_up, 1u);
       if (with_z) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tbase + SH::ColZ, adv(d_k_mn, 1024 * kk), adv(d_k_mn, 1024 * kk), id_z, 1u);
+          mma_ss(tbase + SH::ColZ, adv(d_k_mn, kvo + 1024 * kk), adv(d_k_mn, kvo + 1024 * kk), id_z, 1u);
       }
     };
 
@@ -477,7 +493,8 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
         if (ok) ok = update_round(IC<2>{});
       }
       if (!ok) break;
-      if (threadIdx.x == 0 && i + 1 < nchunks) load_kv(i + 1);       // K, V no longer read
+      // this stage's K, V are no longer read: chunk i + 2 goes into it
+      if (threadIdx.x == 0 && i + 2 < nchunks) load_kv(i + 2);
       continue;
     } else {
       if (!(ok = wait_all(&bars[kVBarLoadQ], i & 1))) break;
