@@ -269,12 +269,10 @@ KATA_API kata_status_t kata_chunked_state(const void *k, const void *v, int B, i
  *  - Returns KATA_ERR_WORKSPACE, before launching anything, when the problem
  *    needs more scratch than the array holds, i.e. when
  *    kata_fwd_chunked_workspace_bytes(...) > KATA_NOALLOC_SCRATCH_BYTES.
- *  - The first call on a device looks up the array's device address for that
- *    device (cudaGetSymbolAddress with the device current); make that first
- *    call before any stream capture. The address is kept for the life of the
- *    process: after cudaDeviceReset (or anything else that destroys the
- *    device's primary context) it is stale, so do not call this entry point
- *    on that device again in the same process.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress), so a cudaDeviceReset or a new primary context
+ *    leaves no stale address behind. The first call on a device may load the
+ *    library's device code: make it before any stream capture.
  *  - All calls share the array, which keeps the last call's contents (each
  *    call clears the status word it needs to start at zero). Calls whose work
  *    overlaps on the GPU (different streams, different host threads) race on

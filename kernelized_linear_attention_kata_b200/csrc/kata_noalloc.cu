@@ -10,36 +10,28 @@
 // GPU loading this library holds until the process exits.
 //
 // The array's name, used in host code, is only a host-side stand-in for the
-// symbol, not a device address; its device address is looked up once per
-// device with cudaGetSymbolAddress (with that device current) and passed on
-// as the workspace pointer. Every call shares the array: the status word is
+// symbol, not a device address; its device address on the current device is
+// looked up with cudaGetSymbolAddress on every call and passed on as the
+// workspace pointer. Every call shares the array: the status word is
 // cleared at the start of each call (the increments are fully written before
 // they are read), and two calls whose work overlaps on the GPU race on it.
 #include "../../include/kata.h"
 
 #include <cuda_runtime.h>
 
-#include <mutex>
 
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[KATA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on `dev` (the current device), looked
-// up on the first call for that device.
-kata_status_t scratch_for_device(int dev, void **out) {
-  if (dev < 0 || dev >= kMaxDevices) return KATA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_setup_mu);
-  if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return KATA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+// Device address of the scratch array on the current device and context.
+// It is looked up on every call (a table lookup in the runtime once the
+// module is loaded), so that a device reset or a new primary context cannot
+// leave a stale address behind.
+kata_status_t scratch_address(void **out) {
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return KATA_ERR_CUDA;
+  *out = p;
   return KATA_OK;
 }
 
@@ -59,10 +51,8 @@ extern "C" kata_status_t kata_fwd_chunked_noalloc(const void *q, const void *k, 
   const size_t need = kata_fwd_chunked_workspace_bytes(B, H, T, d_k, d_v, C, dtype, feature);
   if (need == 0) return KATA_ERR_CUDA;
   if (need > (size_t)KATA_NOALLOC_SCRATCH_BYTES) return KATA_ERR_WORKSPACE;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KATA_ERR_CUDA;
   void *scratch = nullptr;
-  const kata_status_t st = scratch_for_device(dev, &scratch);
+  const kata_status_t st = scratch_address(&scratch);
   if (st != KATA_OK) return st;
   return kata_fwd_chunked(q, k, v, o, B, H, T, d_k, d_v, C, dtype, feature, S_out, z_out, scratch,
                           (size_t)KATA_NOALLOC_SCRATCH_BYTES, stream);
