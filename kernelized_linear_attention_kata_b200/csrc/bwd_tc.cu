@@ -520,7 +520,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
         const float m1 = s0 + 2 * j + 1 <= r ? 2.f * a1 * e1 : 0.f;
         m[j] = pack_bf16x2(m0, m1);
       }
-      if (b == 0 && upd) write_upd(IC<1>{});   // update round 0 (the last round) read its tiles
+      if (b == 0 && upd) write_upd(IC<1>{});   // the first update (the last MMA round) read its tiles
       __syncthreads();          // every thread has read A and D' before M overwrites A
       tmem_st16(tbase + lane_off + kColA + 16 * half, m);
       ok = round([&](int who) {

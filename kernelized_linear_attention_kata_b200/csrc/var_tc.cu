@@ -33,12 +33,12 @@
 // each round of MMAs (each accumulator's chain from one of them) and commit
 // it to one barrier every thread waits on. Independent MMAs share rounds:
 // per chunk
-//   1: U = Q Zd and the blocks of keys 0..63
-//   2: P V (keys 0..63, P in U's columns), the blocks of keys 64..127,
+//   A: U = Q Zd and the blocks of keys 0..63
+//   B: P V (keys 0..63, P in U's columns), the blocks of keys 64..127,
 //      readout groups 0, 1
-//   3: P V (keys 64..127), readout groups 2 (, 3), the update of state tiles
+//   C: P V (keys 64..127), readout groups 2 (, 3), the update of state tiles
 //      0, 1 and Z
-//   4 (Mg2): readout group 4, the update of tile 2
+//   D (Mg2): readout group 4, the update of tile 2
 // (four rounds for Mg2, three for Sg2), the operands of the next round
 // written by the threads in between.
 //
@@ -567,7 +567,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
       constexpr uint32_t kColP1 = V == kMg2 ? SH::ColW + 128 : SH::ColW;
       static_assert(V != kMg2 || SH::ColW + 160 <= kVTmemCols, "P of the second key half");
 
-      // round 1: U = Q Zd, the blocks of keys 0..63
+      // MMA round A: U = Q Zd, the blocks of keys 0..63
       ok = round([&](int who) {
         if (who == 0) {
 #pragma unroll
@@ -597,7 +597,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
         tmem_st16(tbase + lane_off + SH::ColU + 16 * half, p);
       }
       if (half) slot_group(IC<1>{}); else slot_group(IC<0>{});
-      // round 2: P V (keys 0..63), the blocks of keys 64..127, readout groups 0, 1
+      // MMA round B: P V (keys 0..63), the blocks of keys 64..127, readout groups 0, 1
       ok = round([&](int who) {
         if (who == 0) {                          // the O accumulator
           issue_pv(0, SH::ColU);
@@ -619,7 +619,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
       if (upd) {
         if (half) tile_groups(IC<1>{}, buf + 32768); else tile_groups(IC<0>{}, buf);
       }
-      // round 3: P V (keys 64..127), readout groups 2, 3, update of tiles 0, 1 and Z
+      // MMA round C: P V (keys 64..127), readout groups 2, 3, update of tiles 0, 1 and Z
       ok = round([&](int who) {
         if (who == 0) {                          // O, and state tile 1
           issue_pv(1, kColP1);
@@ -632,7 +632,7 @@ var_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ C
       });
       if (!ok) break;
       if constexpr (NG > 4) {
-        // round 4 (Mg2): readout group 4, update of tile 2
+        // MMA round D (Mg2): readout group 4, update of tile 2
         if (!half) slot_group(IC<4>{});
         if (upd && !half) tile_groups(IC<2>{}, buf);
         ok = round([&](int who) {
