@@ -460,23 +460,23 @@ def run_ours(args, rank, world, local_rank):
             nb = api.bwd_chunked_workspace_bytes(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature)
             ws = torch.empty(nb, dtype=torch.uint8, device=dev)
 
-            def step():
-                api.kata_bwd_chunked(q, k, v, dy, dq, dk, dv, w.C, w.feature, workspace=ws)
+            def run_on(ins, outs):
+                api.kata_bwd_chunked(*ins, *outs, w.C, w.feature, workspace=ws)
             flops_th, bytes_th = algorithmic_backward_per_token_head(w.d_k, w.d_v, w.C, w.feature)
             e2e_in, e2e_out = [q, k, v, dy], [dq, dk, dv]
         elif form == "delta":
             beta = W.make_delta_beta(w.B, w.H, w.T, w.seed, device=dev)
             ws = torch.empty(256, dtype=torch.uint8, device=dev)
 
-            def step():
-                api.kata_fwd_delta(q, k, v, beta, o, w.feature, workspace=ws)
+            def run_on(ins, outs):
+                api.kata_fwd_delta(*ins, beta, *outs, w.feature, workspace=ws)
             flops_th, bytes_th = algorithmic_delta_per_token_head(w.d_k, w.d_v)
             phi_th = 3 * state_rows(w.d_k, "psd")
         elif form == "quadratic":
             ws = None
 
-            def step():
-                api.kata_fwd_quadratic(q, k, v, o, w.feature)
+            def run_on(ins, outs):
+                api.kata_fwd_quadratic(*ins, *outs, w.feature)
             flops_th = (w.T + 1) / 2 * (2 * w.d_k + 2 * w.d_v + 2)
             _, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
         elif seq:
@@ -489,18 +489,23 @@ def run_ours(args, rank, world, local_rank):
             w = w.with_T(Tr)
             ws = None
 
-            def step():
-                SP.fwd_chunked_sequence_parallel(q, k, v, w.C, w.feature, out=o)
+            def run_on(ins, outs):
+                SP.fwd_chunked_sequence_parallel(*ins, w.C, w.feature, out=outs[0])
             flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
             phi_th = feature_products_per_token_head(w.d_k, w.feature)
         else:
             ws = api.alloc_workspace(w.B, w.H, w.T, w.d_k, w.d_v, w.C, q.dtype, w.feature, dev)
             seq_carry = form in ("sequential", "first_order_sequential")
 
-            def step():
-                api.kata_fwd_chunked(q, k, v, o, w.C, w.feature, workspace=ws, sequential=seq_carry)
+            def run_on(ins, outs):
+                api.kata_fwd_chunked(*ins, *outs, w.C, w.feature, workspace=ws, sequential=seq_carry)
             flops_th, bytes_th = algorithmic_per_token_head(w.d_k, w.d_v, w.C, w.feature)
             phi_th = feature_products_per_token_head(w.d_k, w.feature)
+        if form != "backward":
+            e2e_in, e2e_out = [q, k, v], [o]
+
+        def step():
+            run_on(e2e_in, e2e_out)
         tokens_per_step = w.B * w.T
         token_heads = w.B * w.H * w.T
         config = workload_config(w)
@@ -587,37 +592,44 @@ def run_ours(args, rank, world, local_rank):
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e and form != "decode":
-        if form != "backward":
-            e2e_in, e2e_out = [q, k, v], [o]
         hosts_in = [t.cpu().pin_memory() for t in e2e_in]
         hosts_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in e2e_out]
 
         # A serving loop: step i's inputs go in on one copy stream, its result
-        # comes back on another, so that the two directions of the link
-        # overlap across steps; each step's compute waits for its own inputs
-        # and for the previous result to have left its output buffers.
+        # comes back on another, and the device buffers alternate between two
+        # sets, so that step i + 1's inputs cross the link while step i
+        # computes and step i - 1's result leaves. Each step's compute waits
+        # for its own inputs and for the result last computed in its buffer
+        # set (two steps back) to have left; each copy in waits for the
+        # compute that last read its buffer set.
+        ins_sets = [e2e_in, [torch.empty_like(t) for t in e2e_in]]
+        outs_sets = [e2e_out, [torch.empty_like(t) for t in e2e_out]]
         h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-        last = {"compute": None, "out": None}
+        last = [{"compute": None, "out": None}, {"compute": None, "out": None}]
+        count = [0]
 
         def e2e_step():
+            b = count[0] % 2
+            count[0] += 1
+            ins, outs = ins_sets[b], outs_sets[b]
             ev_in, ev_comp, ev_out = (torch.cuda.Event() for _ in range(3))
             with torch.cuda.stream(h2d_s):
-                if last["compute"] is not None:
-                    h2d_s.wait_event(last["compute"])          # inputs no longer read
-                for d, h in zip(e2e_in, hosts_in):
+                if last[b]["compute"] is not None:
+                    h2d_s.wait_event(last[b]["compute"])       # this set's inputs no longer read
+                for d, h in zip(ins, hosts_in):
                     d.copy_(h, non_blocking=True)
                 ev_in.record(h2d_s)
             stream.wait_event(ev_in)
-            if last["out"] is not None:
-                stream.wait_event(last["out"])                 # outputs copied out
-            step()
+            if last[b]["out"] is not None:
+                stream.wait_event(last[b]["out"])              # this set's outputs copied out
+            run_on(ins, outs)
             ev_comp.record(stream)
             with torch.cuda.stream(d2h_s):
                 d2h_s.wait_event(ev_comp)
-                for h, d in zip(hosts_out, e2e_out):
+                for h, d in zip(hosts_out, outs):
                     h.copy_(d, non_blocking=True)
                 ev_out.record(d2h_s)
-            last["compute"], last["out"] = ev_comp, ev_out
+            last[b] = {"compute": ev_comp, "out": ev_out}
 
         for _ in range(2):
             e2e_step()
@@ -636,7 +648,8 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in e2e_in),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in e2e_out),
                "ms_per_step": ms_e2e,
-               "overlap": "step i+1 in and step i out on separate copy streams"}
+               "overlap": "two device buffer sets: step i+1 in, step i computing and step i-1 "
+                          "out at once, on two copy streams and the compute stream"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and form == "chunked":
