@@ -105,20 +105,46 @@ delta_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__
   }
   const size_t qoff = (size_t)bh * T * DK, voff = (size_t)bh * T * DV;
 
+  // The inputs of a chunk are fetched into registers one chunk ahead (their
+  // global-memory latency hides behind the previous chunk's three phases)
+  // and moved to shared memory at the chunk's start.
+  constexpr int NQK = (kDC * DK + kDelThreads - 1) / kDelThreads;   // q, k values a thread
+  static_assert(kDC * kCG <= kDelThreads && kDC <= kDelThreads, "one v value and one beta a thread");
+  float pq[NQK], pk[NQK], pv = 0.f, pb = 0.f;
+  auto fetch = [&](int tc) {                    // chunk starting at token tc
+    const int nn = min(kDC, T - tc);
+#pragma unroll
+    for (int j = 0; j < NQK; ++j) {
+      const int e = tid + j * kDelThreads;
+      const int t = e / DK, i = e % DK;
+      const bool in = e < kDC * DK && t < nn;
+      pq[j] = in ? to_f(q[qoff + (size_t)(tc + t) * DK + i]) : 0.f;
+      pk[j] = in ? to_f(k[qoff + (size_t)(tc + t) * DK + i]) : 0.f;
+    }
+    if (tid < kDC * kCG) {
+      const int t = tid / kCG, c = tid % kCG;
+      pv = t < nn ? to_f(v[voff + (size_t)(tc + t) * DV + c0 + c]) : 0.f;
+    }
+    if (tid < kDC) pb = tid < nn ? beta[(size_t)bh * T + tc + tid] : 0.f;
+  };
+  if (T > 0) fetch(0);
+
   for (int t0 = 0; t0 < T; t0 += kDC) {
     const int n = min(kDC, T - t0);
     __syncthreads();                            // previous chunk's readers are done
-    for (int e = tid; e < kDC * DK; e += kDelThreads) {
-      const int t = e / DK, i = e % DK;
-      qs[t * KS + i] = t < n ? to_f(q[qoff + (size_t)(t0 + t) * DK + i]) : 0.f;
-      ks[t * KS + i] = t < n ? to_f(k[qoff + (size_t)(t0 + t) * DK + i]) : 0.f;
+#pragma unroll
+    for (int j = 0; j < NQK; ++j) {
+      const int e = tid + j * kDelThreads;
+      if (e < kDC * DK) {
+        const int t = e / DK, i = e % DK;
+        qs[t * KS + i] = pq[j];
+        ks[t * KS + i] = pk[j];
+      }
     }
-    for (int e = tid; e < kDC * kCG; e += kDelThreads) {
-      const int t = e / kCG, c = e % kCG;
-      vs[e] = t < n ? to_f(v[voff + (size_t)(t0 + t) * DV + c0 + c]) : 0.f;
-    }
-    if (tid < kDC) bs[tid] = tid < n ? beta[(size_t)bh * T + t0 + tid] : 0.f;
+    if (tid < kDC * kCG) vs[tid] = pv;
+    if (tid < kDC) bs[tid] = pb;
     __syncthreads();
+    if (t0 + kDC < T) fetch(t0 + kDC);          // the next chunk, in flight during this one
 
     // ---- phase 1: partial phi~(k_t)^T S'_0, phi~(q_t)^T S'_0 over rows r = warp mod 16 ----
     {
