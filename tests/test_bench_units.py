@@ -52,3 +52,20 @@ def test_floors_order_on_the_long_workload():
     assert 115e-6 < t_hbm < 125e-6
     assert 55e-6 < t_alu < 65e-6
     assert t_tensor > t_hbm > t_alu
+
+
+def test_traffic_records_match_the_current_sources():
+    """Every DRAM-traffic record in profiles/traffic.json names a kernel the
+    bench knows, holds a positive byte count, and is keyed to the hash of
+    that kernel's current source files: a kernel edited after its capture
+    must be profiled again (the bench would otherwise report its traffic as
+    unknown)."""
+    import json
+    b = bench()
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        records = json.load(f)
+    assert records
+    for kernel, rec in records.items():
+        assert kernel in b.KERNEL_SOURCES, kernel
+        assert rec["bytes_per_launch"] > 0, kernel
+        assert rec["source_sha"] == b.source_hash(kernel), f"{kernel}: captured on other sources"
