@@ -375,37 +375,39 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
     }
     if (half) rot<8>(qR);
     float dn_car = 0.f;
-    for (int j = 0; ok && j < 5; ++j) {
+    // four rounds; the last also takes the 16 features of tile 4 (half 1's)
+    // into the dq columns, free between the read of U and the first dq MMA
+    for (int j = 0; ok && j < 4; ++j) {
       ok = round([&](int who) {
-        if (j < 4 && who == 0) {
+        if (who == 0) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tbase + kColA, adv(d_o, 32 * kk), adv(d_snap, 64 * j * 128 + 32 * kk), id_n64, kk);
-        } else if (j < 4) {
+        } else {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_snap, (256 + 64 * j) * 128 + 32 * kk),
                    id_n64, kk);
-        } else if (who == 1) {
+          if (j == 3) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tbase + kColB, adv(d_o, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tbase + kColDq, adv(d_o, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
+          }
         }
       });
       if (!ok) break;
-      if (j < 4) {
-        uint32_t x[32];
-        tmem_ld32(tbase + lane_off + kColA + 64 * half, x);
+      uint32_t x[32];
+      tmem_ld32(tbase + lane_off + kColA + 64 * half, x);
+      tmem_wait_ld();
+      contract_offset<32>(x, q, qR, h, g2R, dn_car);
+      tmem_ld32(tbase + lane_off + kColA + 64 * half + 32, x);
+      tmem_wait_ld();
+      contract_offset<32>(x, q, qR, h, g2R, dn_car);
+      if (j == 3 && half) {
+        uint32_t x16[16];
+        tmem_ld16(tbase + lane_off + kColDq, x16);
         tmem_wait_ld();
-        contract_offset<32>(x, q, qR, h, g2R, dn_car);
-        tmem_ld32(tbase + lane_off + kColA + 64 * half + 32, x);
-        tmem_wait_ld();
-        contract_offset<32>(x, q, qR, h, g2R, dn_car);
-      } else if (half) {
-        uint32_t x[16];
-        tmem_ld16(tbase + lane_off + kColB, x);
-        tmem_wait_ld();
-        contract_offset<16>(x, q, qR, h, g2R, dn_car);
+        contract_offset<16>(x16, q, qR, h, g2R, dn_car);
       }
     }
     if (!ok) break;
@@ -899,27 +901,31 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
       }
       if (half) rot<8>(kR);
       float unused = 0.f;
-      for (int j = 0; ok && j < 5; ++j) {
+      // four rounds; the last also takes the 16 features of tile 4 (half
+      // 1's) into the dk columns, free between the read of U2 and the first
+      // dk MMA
+      for (int j = 0; ok && j < 4; ++j) {
         ok = round([&](int who) {
           if (j == 0 && who == 0) {
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk)
               mma_ss(tbase + kColDk, adv(d_k, 32 * kk), adv(d_rq, 32 * kk), id_n32, kk);
           }
-          if (j < 4 && who == 0) {
+          if (who == 0) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_ss(tbase + kColDv, adv(d_v, 32 * kk), adv(d_snap, 64 * j * 128 + 32 * kk), id_n64,
                      kk);
-          } else if (j < 4) {
+          } else {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_ss(tbase + kColW, adv(d_v, 32 * kk), adv(d_snap, (256 + 64 * j) * 128 + 32 * kk),
                      id_n64, kk);
-          } else if (who == 1) {
+            if (j == 3) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ss(tbase + kColW, adv(d_v, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tbase + kColDk, adv(d_v, 32 * kk), adv(d_snap, 512 * 128 + 32 * kk), id_n16, kk);
+            }
           }
         });
         if (!ok) break;
@@ -933,7 +939,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
                 make_float4(__uint_as_float(u[l]), __uint_as_float(u[l + 1]),
                             __uint_as_float(u[l + 2]), __uint_as_float(u[l + 3]));
         }
-        if (j < 4) {
+        {
           uint32_t x[32];
           const uint32_t col = half ? kColW : kColDv;
           tmem_ld32(tbase + lane_off + col, x);
@@ -942,11 +948,12 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
           tmem_ld32(tbase + lane_off + col + 32, x);
           tmem_wait_ld();
           contract_offset<32, false>(x, kf, kR, h, g2R, unused);
-        } else if (half) {
-          uint32_t x[16];
-          tmem_ld16(tbase + lane_off + kColW, x);
+        }
+        if (j == 3 && half) {
+          uint32_t x16[16];
+          tmem_ld16(tbase + lane_off + kColDk, x16);
           tmem_wait_ld();
-          contract_offset<16, false>(x, kf, kR, h, g2R, unused);
+          contract_offset<16, false>(x16, kf, kR, h, g2R, unused);
         }
       }
       if (!ok) break;
